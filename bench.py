@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Throughput of one FOCUS focused denoising step on B200: decoded tokens/s, step latency, roofline.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+One "step" is one pass of the whole focused step (embed, layers 0-1 with importance, delta / budget /
+top-k, compaction, layers 2..L-1 on the kept rows, LM head + decode) over one batch.  The default
+workload is the SDAR-1.7B-shaped random-init bf16 model with 32 ragged requests, block 32, prefixes
+U[256, 1024] in 64-token pages, masked fraction U[0.3, 1.0], k_max 8.  Under torchrun each rank runs an
+independent replica on its own 32 requests (requests are independent: no collective on the data
+path), so the scaling is weak.
+
+`--impl reference` times the CPU oracle (test infrastructure, float64 numpy) on the host cores instead,
+one request of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import focus_synth as fs  # noqa: E402
+
+METRIC = "decoded tokens/s per focused step on 1 B200; step latency; % of roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["focus", "reference"], default="focus")
+    ap.add_argument("--workload", default="sdar1.7b_n32_b32")
+    ap.add_argument("--roofline-kernel", default="auto", help="kernel class for the roofline (default: dominant)")
+    ap.add_argument("--cpu-baseline-requests", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def workload_desc(case: fs.Case) -> str:
+    s, w = case.shape, case.work
+    return (f"{s.n_layers}L D{s.hidden} {s.n_q_heads}/{s.n_kv_heads} heads d{s.head_dim} F{s.ffn} V{s.vocab} {s.dtype}; "
+            f"N={w.n_requests} B={w.block} prefix {w.prefix} page {w.page_size} masked {w.masked} "
+            f"k_min {w.k_min} k_max {w.k_max} tau {w.tau} threshold {w.conf_threshold}")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            d = json.load(open(p))
+            return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+        except Exception:
+            pass
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "50", "-i", uuid], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self, t0, t1):
+        rows = [r for t, r in self.samples if t0 <= t <= t1 + 0.06]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no sample inside the timed region"],
+                    "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        mx = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[6:10]) if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((num(r[4]) or 0.0) for r in rows)}
+
+
+# ------------------------------------------------------------------ roofline bookkeeping
+def algorithmic_work(kclass: str, case: fs.Case, R: int, kept_per_req, plen, splits=1):
+    """(bytes, flops) one launch of `kclass` must move / compute at the minimum (bf16 operands)."""
+    s = case.shape
+    D, F, V, Hq, Hkv, d = s.hidden, s.ffn, s.vocab, s.n_q_heads, s.n_kv_heads, s.head_dim
+    qkv = (Hq + 2 * Hkv) * d
+    N, B = case.work.n_requests, case.work.block
+    e = 2
+    full = kclass.startswith("gemm_full")
+    M = N * B if full else R
+    gem = {"qkv": (qkv, D, M * qkv * 4), "o": (D, Hq * d, M * D * 4), "gateup": (2 * F, D, M * F * e),
+           "down": (D, F, M * D * 4), "lmhead": (V, D, 0)}
+    for key, (n, k, out_bytes) in gem.items():
+        if kclass.endswith("_" + key) or kclass == "gemm_" + key:
+            return n * k * e + M * k * e + out_bytes, 2.0 * M * n * k
+    if kclass in ("attn_score", "attn_ragged"):
+        rows = [B] * N if kclass == "attn_score" else list(kept_per_req)
+        by = fl = 0.0
+        for b in range(N):
+            if rows[b] == 0:
+                continue
+            keys = int(plen[b]) + B
+            by += keys * Hkv * d * e * 2 + rows[b] * Hq * d * e * 2
+            fl += 4.0 * rows[b] * Hq * d * keys
+        return by, fl
+    return None, None
+
+
+def source_digest(kclass: str) -> str:
+    files = {"gemm": ["tc_gemm.cu", "gemm_simt.cu"], "attn": ["attention.cu"], "row": ["rows.cu"],
+             "qkv": ["rows.cu"], "embed": ["rows.cu"], "select": ["select.cu"], "decode": ["decode.cu"]}
+    key = kclass.split("_")[0]
+    h = hashlib.sha256()
+    for f in files.get(key, []):
+        p = os.path.join(ROOT, "decodability_aware_token_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kclass: str):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        ent = json.load(open(p)).get(kclass)
+    except Exception:
+        return None
+    if not ent or ent.get("source_digest") != source_digest(kclass):
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ CPU oracle timings
+def oracle_tokens_per_s(case_host: fs.Case, requests, model=None):
+    from oracle import focus_oracle as fo
+    w = case_host.work
+    t0 = time.perf_counter()
+    r = fo.focus_step(case_host.shape, model if model is not None else case_host.model, case_host.batch, tau=w.tau,
+                      k_min=w.k_min, k_max=w.k_max, conf_threshold=w.conf_threshold, alpha=w.alpha,
+                      forced_keep_frac=w.forced_keep_frac, requests=list(requests))
+    dt = time.perf_counter() - t0
+    return int((r.decoded_ids >= 0).sum()), dt
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args):
+    """The oracle on the host cores: each step is one request of the workload (requests cycle)."""
+    case = fs.make_case(args.workload)
+    model64 = {k: ([t.to(torch.float64).numpy() for t in v] if isinstance(v, list) else v.to(torch.float64).numpy())
+               for k, v in case.model.items()}
+    N = case.work.n_requests
+    for i in range(args.warmup):
+        oracle_tokens_per_s(case, [i % N], model64)
+    tok, secs = 0, 0.0
+    for i in range(args.steps):
+        t, dt = oracle_tokens_per_s(case, [(args.warmup + i) % N], model64)
+        tok += t
+        secs += dt
+    value = tok / secs if secs > 0 else 0.0
+    cores = blas_threads()
+    sample = (f"one of {N} requests per step (cycling), float64 oracle, weights converted to float64 once "
+              f"before the timed steps")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "desc": workload_desc(case), "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ the GPU arm
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+    import torch.distributed as dist
+    from decodability_aware_token_b200 import FocusContext, StepParams, StepOutputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    base = fs.SEEDS.get(args.workload, 1234)
+    case = fs.make_case(args.workload, seed=base + 7919 * rank, device=dev)    # this rank's requests
+    w, shp = case.work, case.shape
+    N, B = w.n_requests, w.block
+    params = StepParams(w.tau, w.k_min, w.k_max, w.conf_threshold, w.alpha, w.forced_keep_frac)
+    mk = B if w.forced_keep_frac >= 0 else w.k_max
+    ctx = FocusContext(shp, case.model, max_requests=N, max_block=B, max_keep=mk,
+                       max_pages_per_req=case.max_pages_per_req)
+    K, Wm = args.steps, max(3, args.warmup)
+    tok0, mask0, ibc0 = case.batch["block_tokens"], case.batch["mask"], case.batch["ibc"]
+
+    def fresh_state():
+        b = dict(case.batch)
+        b["block_tokens"], b["mask"], b["ibc"] = tok0.clone(), mask0.clone(), ibc0.clone()
+        return b
+
+    # every step gets the workload's initial state (a step decodes in place, which would shrink later steps)
+    states = [fresh_state() for _ in range(Wm + K)]
+    outs = [StepOutputs.alloc(N, B, mk, shp.hidden, dev, importance=False, hidden=False) for _ in range(Wm + K)]
+    stream = torch.cuda.current_stream(dev)
+
+    for i in range(Wm):
+        ctx.step(states[i], params, outs[i])
+    torch.cuda.synchronize(dev)
+    launches_per_step = ctx.last_step_launches()
+    kept = outs[0].keep_count.cpu()
+    R = int(kept.sum())
+    plen = case.batch["prefix_len"].cpu()
+
+    # which kernel class dominates (a few untimed steps per class, then fresh states again)
+    from decodability_aware_token_b200 import _abi
+    per_class = {}
+    if args.roofline_kernel == "auto":
+        probe = fresh_state()
+        for kc in _abi.KERNEL_CLASSES:
+            ctx.profile_begin(kc, 4096)
+            for _ in range(2):
+                probe["block_tokens"].copy_(tok0); probe["mask"].copy_(mask0); probe["ibc"].copy_(ibc0)
+                ctx.step(probe, params, outs[0])
+            ms, n = ctx.profile_end()
+            per_class[kc] = (ms / 2.0, n / 2.0)
+        roof_class = max(per_class, key=lambda k: per_class[k][0])
+        del probe
+    else:
+        roof_class = args.roofline_kernel
+    torch.cuda.synchronize(dev)
+
+    # ---- timed region: device events on the launching stream, max over ranks
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ctx.profile_begin(roof_class, max(1, K * 64))
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tw0 = time.time()
+    ev0.record(stream)
+    for i in range(K):
+        ctx.step(states[Wm + i], params, outs[Wm + i])
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    tw1 = time.time()
+    kern_ms, kern_n = ctx.profile_end()
+    barrier()
+    time.sleep(0.1)
+    sampler.stop()
+    clocks = sampler.summary(tw0, tw1)
+    elapsed = ev0.elapsed_time(ev1)
+    decoded = sum(int((o.decoded_ids >= 0).sum()) for o in outs[Wm:])
+    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+    tk = torch.tensor([decoded], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(tk, op=dist.ReduceOp.SUM)
+    max_ms, total_decoded = float(t.item()), float(tk.item())
+    value = total_decoded / (max_ms / 1e3)
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        host_in = {k: case.batch[k].cpu().pin_memory() for k in ("block_tokens", "mask", "prefix_len", "page_table")}
+        host_in["block_tokens"].copy_(tok0.cpu())
+        host_in["mask"].copy_(mask0.cpu())
+        for st in states:
+            st["ibc"].copy_(ibc0)
+        outs_h = [StepOutputs.alloc(N, B, mk, shp.hidden, "cpu", importance=False, hidden=False, pin_memory=True)
+                  for _ in range(K)]
+        h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+        d2h = sum(getattr(outs_h[0], k).numel() * getattr(outs_h[0], k).element_size()
+                  for k in ("keep_count", "retained_idx", "decoded_ids", "conf", "top_id"))
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(K):
+            st = states[Wm + i]
+            for k_, v in host_in.items():
+                st[k_].copy_(v, non_blocking=True)
+            o = ctx.step(st, params, outs[Wm + i])
+            for k_ in ("keep_count", "retained_idx", "decoded_ids", "conf", "top_id"):
+                getattr(outs_h[i], k_).copy_(getattr(o, k_), non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        e_dec = sum(int((o.decoded_ids >= 0).sum()) for o in outs_h)
+        te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        tke = torch.tensor([e_dec], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+            dist.all_reduce(tke, op=dist.ReduceOp.SUM)
+        e2e = {"value": float(tke.item()) / (float(te.item()) / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+
+    # ---- roofline of the dominant kernel class
+    peaks, peak_src = load_peaks()
+    by, fl = algorithmic_work(roof_class, case, R, kept.tolist(), plen.tolist())
+    roofline = None
+    if by is not None and kern_n > 0:
+        avg_s = kern_ms / kern_n / 1e3
+        t_b = by / (peaks["hbm_gbs"] * 1e9)
+        t_f = fl / (peaks["bf16_tflops_sustained"] * 1e12)
+        if t_f > t_b:
+            ach = fl / avg_s / 1e12
+            roofline = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                        "frac": ach / peaks["bf16_tflops_sustained"]}
+        else:
+            ach = by / avg_s / 1e9
+            roofline = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": ach / peaks["hbm_gbs"]}
+        roofline.update({"traffic": recorded_traffic(roof_class), "kernel": roof_class,
+                         "peak_source": f"{peak_src} ({'sustained bf16' if roofline['bound'] == 'tensor' else 'HBM copy'})",
+                         "launches_timed": kern_n, "avg_launch_us": avg_s * 1e6,
+                         "algorithmic_bytes_per_launch": by, "algorithmic_flops_per_launch": fl,
+                         "kept_rows": R})
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = fs.Case(shp, w, {k: ([x.cpu() for x in v] if isinstance(v, list) else v.cpu())
+                                for k, v in case.model.items()},
+                       {k: v.cpu() for k, v in case.batch.items()}, case.seed)
+        host.batch["block_tokens"], host.batch["mask"], host.batch["ibc"] = tok0.cpu(), mask0.cpu(), ibc0.cpu()
+        nreq = min(N, args.cpu_baseline_requests)
+        ctok, csec = oracle_tokens_per_s(host, range(nreq))
+        cpu = {"value": ctok / csec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{nreq} of {N} requests of the same batch, one oracle call ({csec:.1f} s, "
+                         f"float64, weight conversion included)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm,
+            "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if shp.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": args.workload, "desc": workload_desc(case), "requests_per_gpu": N,
+                       "global_batch": N * world, "block": B, "kept_rows_per_step": R,
+                       "decoded_per_step": total_decoded / K / world,
+                       "l2": "inputs larger than L2 (3.4 GB of weights and ~2.4 GB of KV pages streamed per step)",
+                       "parallelism": f"replicas x{world} (requests sharded, no collective)"},
+            "gpu_launches": launches_per_step * K,
+            "clocks": clocks, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "per_class_ms_per_step": {k: round(v[0], 4) for k, v in per_class.items()} if per_class else None,
+        }
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

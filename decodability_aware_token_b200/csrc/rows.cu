@@ -1,0 +1,160 @@
+// Row-wise kernels of the step: embedding + RMSNorm, residual reduction + RMSNorm (optionally
+// gathering the kept rows), and the QKV finalisation (RoPE + intra-block KV-cache write).
+// All three are HBM-bound row sweeps: one CTA per row, coalesced loads, fixed-order reductions.
+#include "launch.h"
+
+namespace focus {
+
+namespace {
+
+constexpr int kRowThreads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) embed_norm_kernel(const int32_t* __restrict__ tokens, int V,
+                                                                 const T* __restrict__ embed,
+                                                                 const T* __restrict__ gamma, float eps, int D,
+                                                                 float* __restrict__ x, T* __restrict__ h,
+                                                                 int* err) {
+    __shared__ float red[32];
+    const int r = blockIdx.x;
+    int tok = tokens[r];
+    if (tok < 0 || tok >= V) {
+        if (threadIdx.x == 0) raise_err(err, FOCUS_DEVERR_TOKEN_ID);
+        tok = 0;
+    }
+    const T* e = embed + (size_t)tok * D;
+    float* xr = x + (size_t)r * D;
+    float ss = 0.f;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+        float v = to_f(e[i]);
+        xr[i] = v;
+        ss += v * v;
+    }
+    const float tot = block_sum(ss, red);
+    const float inv = rsqrtf(tot / D + eps);
+    T* hr = h + (size_t)r * D;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) hr[i] = from_f<T>(xr[i] * inv * to_f(gamma[i]));
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) residual_norm_kernel(
+    const float* __restrict__ x_in, const int32_t* __restrict__ src_map, const int32_t* __restrict__ n_rows_dev,
+    const float* __restrict__ part, int n_splits, size_t part_stride, float* x_out, const T* __restrict__ gamma,
+    float eps, int D, T* __restrict__ h_out) {
+    __shared__ float red[32];
+    const int r = blockIdx.x;
+    if (n_rows_dev && r >= *n_rows_dev) return;
+    const int src = src_map ? src_map[r] : r;
+    const float* xi = x_in + (size_t)src * D;
+    float* xo = x_out + (size_t)r * D;
+    float ss = 0.f;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+        float v = xi[i];
+        for (int s = 0; s < n_splits; ++s) v += part[(size_t)s * part_stride + (size_t)src * D + i];
+        xo[i] = v;
+        ss += v * v;
+    }
+    if (!h_out) return;
+    const float tot = block_sum(ss, red);
+    const float inv = rsqrtf(tot / D + eps);
+    T* hr = h_out + (size_t)r * D;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) hr[i] = from_f<T>(xo[i] * inv * to_f(gamma[i]));
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) qkv_finalize_kernel(const float* __restrict__ part, int n_splits,
+                                                                   size_t part_stride, RowMap rm,
+                                                                   const int32_t* __restrict__ prefix_len,
+                                                                   int max_prefix, const double* __restrict__ inv_freq,
+                                                                   Dims dm, int layer, T* __restrict__ q_out,
+                                                                   T* __restrict__ ibc, int* err) {
+    extern __shared__ float cs[];  // [d/2] cos, [d/2] sin
+    const int r = blockIdx.x;
+    if (r >= rm.rows()) return;
+    int b, j;
+    rm.coords(r, b, j);
+    const int d = dm.d, half = d / 2;
+    const int P = checked_prefix(prefix_len, b, max_prefix, err);
+    const double pos = (double)(P + j);
+    for (int i = threadIdx.x; i < half; i += blockDim.x) {
+        double sn, cn;
+        sincos(pos * inv_freq[i], &sn, &cn);
+        cs[i] = (float)cn;
+        cs[half + i] = (float)sn;
+    }
+    __syncthreads();
+    const int B = rm.block;
+    const float* pr = part + (size_t)r * dm.qkv;
+    auto col = [&](int c) {
+        float v = pr[c];
+        for (int s = 1; s < n_splits; ++s) v += pr[(size_t)s * part_stride + c];
+        return v;
+    };
+    // rotated heads: Hq query heads then Hkv key heads, one (i, i + d/2) pair per item
+    const int n_rot = (dm.Hq + dm.Hkv) * half;
+    for (int it = threadIdx.x; it < n_rot; it += blockDim.x) {
+        const int head = it / half, i = it - head * half;
+        const int c0 = head * d + i;
+        const float a = col(c0), bb = col(c0 + half);
+        const float cn = cs[i], sn = cs[half + i];
+        const float lo = a * cn - bb * sn, hi = bb * cn + a * sn;
+        if (head < dm.Hq) {
+            T* qr = q_out + (size_t)r * dm.Hq * d + head * d;
+            qr[i] = from_f<T>(lo);
+            qr[i + half] = from_f<T>(hi);
+        } else {
+            const int g = head - dm.Hq;
+            T* kr = ibc + ((((size_t)b * dm.L + layer) * 2 + 0) * dm.Hkv + g) * B * d + (size_t)j * d;
+            kr[i] = from_f<T>(lo);
+            kr[i + half] = from_f<T>(hi);
+        }
+    }
+    const int n_v = dm.Hkv * d;
+    for (int it = threadIdx.x; it < n_v; it += blockDim.x) {
+        const int g = it / d, i = it - g * d;
+        T* vr = ibc + ((((size_t)b * dm.L + layer) * 2 + 1) * dm.Hkv + g) * B * d + (size_t)j * d;
+        vr[i] = from_f<T>(col((dm.Hq + dm.Hkv) * d + it));
+    }
+}
+
+}  // namespace
+
+template <typename T>
+int launch_embed_norm(const int32_t* tokens, int rows, int V, const T* embed, const T* gamma, float eps, int D,
+                       float* x, T* h, int* err, cudaStream_t s) {
+    if (rows <= 0) return 0;
+    embed_norm_kernel<T><<<rows, kRowThreads, 0, s>>>(tokens, V, embed, gamma, eps, D, x, h, err);
+    return 1;
+}
+
+template <typename T>
+int launch_residual_norm(const float* x_in, const int32_t* src_map, const int32_t* n_rows_dev, int rows_bound,
+                          const float* part, int n_splits, size_t part_stride, float* x_out, const T* gamma,
+                          float eps, int D, T* h_out, cudaStream_t s) {
+    if (rows_bound <= 0) return 0;
+    residual_norm_kernel<T><<<rows_bound, kRowThreads, 0, s>>>(x_in, src_map, n_rows_dev, part, n_splits,
+                                                               part_stride, x_out, gamma, eps, D, h_out);
+    return 1;
+}
+
+template <typename T>
+int launch_qkv_finalize(const float* part, int n_splits, size_t part_stride, RowMap rm, const int32_t* prefix_len,
+                         int max_prefix, const double* inv_freq, Dims dm, int layer, T* q_out, T* ibc, int* err,
+                         cudaStream_t s) {
+    if (rm.rows_static <= 0) return 0;
+    qkv_finalize_kernel<T><<<rm.rows_static, kRowThreads, dm.d * sizeof(float), s>>>(
+        part, n_splits, part_stride, rm, prefix_len, max_prefix, inv_freq, dm, layer, q_out, ibc, err);
+    return 1;
+}
+
+#define FOCUS_INST_ROWS(T)                                                                                         \
+    template int launch_embed_norm<T>(const int32_t*, int, int, const T*, const T*, float, int, float*, T*, int*, \
+                                       cudaStream_t);                                                              \
+    template int launch_residual_norm<T>(const float*, const int32_t*, const int32_t*, int, const float*, int,    \
+                                          size_t, float*, const T*, float, int, T*, cudaStream_t);                 \
+    template int launch_qkv_finalize<T>(const float*, int, size_t, RowMap, const int32_t*, int, const double*,    \
+                                         Dims, int, T*, T*, int*, cudaStream_t);
+FOCUS_INST_ROWS(float)
+FOCUS_INST_ROWS(bf16)
+
+}  // namespace focus

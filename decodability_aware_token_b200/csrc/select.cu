@@ -1,0 +1,152 @@
+// Importance delta -> adaptive budget -> top-k with index tie-break -> ragged row map.
+//
+// "FOCUS: DLLMs Know How to Tame Their Compute Bound", project page, Overview -- Decodability Signal
+// (layer-0-to-1 importance delta), Design (keep likely-decodable candidates under an adaptive budget)
+// and Runtime Action (dynamic budgeting, token eviction, ragged execution); news article on the same
+// paper, "Arquitetura do FOCUS" (target token selection, state compaction).
+//
+// Rules: c = #{masked j : delta_j > tau};  k = min(clamp(ceil(alpha c), k_min, k_max), #masked)
+// (product and ceil in float32); kept = the k best masked positions under (delta desc, j asc),
+// written ascending.  Forced fraction f >= 0: k = min(B, ceil(f B)) over all positions under
+// (masked first, delta desc, j asc).
+//
+// One CTA: a warp per request (B <= 64: each lane owns positions lane and lane + 32), ballots for the
+// counts, an O(B) rank per position (B^2 <= 4096 compares per request), then a serial exclusive scan of
+// the kept counts and the row map.  The work is a few KB, so the kernel is latency-bound by design.
+#include "launch.h"
+
+namespace focus {
+
+namespace {
+
+__device__ __forceinline__ bool key_less(bool forced, bool ma, float da, int ja, bool mb, float db, int jb) {
+    if (forced && ma != mb) return ma;  // masked positions first
+    if (da != db) return da > db;       // larger delta first
+    return ja < jb;                     // lower position first
+}
+
+__global__ void __launch_bounds__(1024) select_kernel(SelectArgs a) {
+    extern __shared__ int32_t sh[];  // [N] kept counts, [N + 1] offsets
+    int32_t* kc_s = sh;
+    int32_t* off_s = sh + a.N;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int B = a.B;
+    const bool forced = a.forced_frac >= 0.f;
+    const size_t layer_stride = (size_t)a.N * a.Hkv * B;
+
+    for (int b = warp; b < a.N; b += nw) {
+        float dl[2];
+        bool valid[2], msk[2], keep[2];
+        for (int h = 0; h < 2; ++h) {
+            const int j = lane + 32 * h;
+            valid[h] = j < B;
+            dl[h] = 0.f;
+            msk[h] = false;
+            if (valid[h]) {
+                float i0 = 0.f, i1 = 0.f;
+                for (int g = 0; g < a.Hkv; ++g) {  // KV groups in order: deterministic
+                    i0 += a.imp_part[((size_t)b * a.Hkv + g) * B + j];
+                    i1 += a.imp_part[layer_stride + ((size_t)b * a.Hkv + g) * B + j];
+                }
+                dl[h] = i1 - i0;
+                msk[h] = a.mask[(size_t)b * B + j] != 0;
+                if (a.importance_out) {
+                    a.importance_out[(size_t)b * B + j] = i0;
+                    a.importance_out[(size_t)a.N * B + (size_t)b * B + j] = i1;
+                }
+            }
+        }
+        if (a.forced_idx) {
+            // caller-chosen set: ascending positions in [0, B), count <= max_keep
+            const int cnt = a.forced_cnt[b];
+            bool bad = cnt < 0 || cnt > a.max_keep || cnt > B;
+            unsigned long long bits = 0ull;
+            if (!bad) {
+                for (int t = lane; t < cnt; t += 32) {
+                    const int j = a.forced_idx[(size_t)b * a.max_keep + t];
+                    const int prev = t > 0 ? a.forced_idx[(size_t)b * a.max_keep + t - 1] : -1;
+                    if (j < 0 || j >= B || j <= prev) bad = true;
+                    else bits |= 1ull << j;
+                }
+            }
+            for (int o = 16; o > 0; o >>= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, o);
+            bad = __any_sync(0xffffffffu, bad);
+            if (bad) {
+                if (lane == 0) raise_err(a.err, FOCUS_DEVERR_FORCED_SET);
+                bits = 0ull;
+            }
+            for (int h = 0; h < 2; ++h) keep[h] = valid[h] && ((bits >> (lane + 32 * h)) & 1ull);
+        } else {
+            bool elig[2];
+            for (int h = 0; h < 2; ++h) elig[h] = valid[h] && (forced || msk[h]);
+            int k;
+            if (forced) {
+                k = min(B, (int)ceilf(a.forced_frac * (float)B));
+            } else {
+                const int c = __popc(__ballot_sync(0xffffffffu, elig[0] && dl[0] > a.tau)) +
+                              __popc(__ballot_sync(0xffffffffu, elig[1] && dl[1] > a.tau));
+                const int n_el = __popc(__ballot_sync(0xffffffffu, elig[0])) + __popc(__ballot_sync(0xffffffffu, elig[1]));
+                k = (int)ceilf(a.alpha * (float)c);
+                k = max(k, a.k_min);
+                k = min(k, a.k_max);
+                k = min(k, n_el);
+            }
+            int rank[2] = {0, 0};
+            for (int jj = 0; jj < B; ++jj) {
+                const int src = jj & 31, hh = jj >> 5;
+                const float d2 = __shfl_sync(0xffffffffu, hh ? dl[1] : dl[0], src);
+                const bool m2 = __shfl_sync(0xffffffffu, (int)(hh ? msk[1] : msk[0]), src) != 0;
+                const bool e2 = __shfl_sync(0xffffffffu, (int)(hh ? elig[1] : elig[0]), src) != 0;
+                for (int h = 0; h < 2; ++h)
+                    if (e2 && key_less(forced, m2, d2, jj, msk[h], dl[h], lane + 32 * h)) ++rank[h];
+            }
+            for (int h = 0; h < 2; ++h) keep[h] = elig[h] && rank[h] < k;
+        }
+        const unsigned lo = __ballot_sync(0xffffffffu, keep[0]);
+        const unsigned hi = __ballot_sync(0xffffffffu, keep[1]);
+        const int kept = __popc(lo) + __popc(hi);
+        const unsigned lt = (1u << lane) - 1u;
+        int32_t* ret = a.retained_idx + (size_t)b * a.max_keep;
+        if (keep[0]) ret[__popc(lo & lt)] = lane;
+        if (keep[1]) ret[__popc(lo) + __popc(hi & lt)] = lane + 32;
+        for (int t = kept + lane; t < a.max_keep; t += 32) ret[t] = -1;
+        if (lane == 0) {
+            a.keep_count[b] = kept;
+            kc_s[b] = kept;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int off = 0;
+        for (int b = 0; b < a.N; ++b) {
+            off_s[b] = off;
+            a.row_offsets[b] = off;
+            off += kc_s[b];
+        }
+        off_s[a.N] = off;
+        a.row_offsets[a.N] = off;
+        *a.n_rows = off;
+    }
+    __syncthreads();
+    for (int b = warp; b < a.N; b += nw) {
+        const int base = off_s[b], k = kc_s[b];
+        for (int t = lane; t < k; t += 32) {
+            const int j = a.retained_idx[(size_t)b * a.max_keep + t];
+            a.row_req[base + t] = b;
+            a.row_pos[base + t] = j;
+            a.row_src[base + t] = b * B + j;
+        }
+    }
+}
+
+}  // namespace
+
+int launch_select(const SelectArgs& a, cudaStream_t s) {
+    if (a.N <= 0) return 0;
+    const size_t smem = sizeof(int32_t) * (2 * (size_t)a.N + 1);
+    if (smem > 48 * 1024) cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    select_kernel<<<1, 1024, smem, s>>>(a);
+    return 1;
+}
+
+}  // namespace focus

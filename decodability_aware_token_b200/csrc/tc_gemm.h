@@ -1,0 +1,30 @@
+// tcgen05 / TMEM / TMA GEMM for the bf16 step: weights' tensor maps are built once at init.
+#pragma once
+#include "launch.h"
+
+namespace focus {
+
+enum WeightId { W_QKV = 0, W_O = 1, W_GATEUP = 2, W_DOWN = 3, W_LM = 4 };
+
+struct TcWeights {
+    int L;
+    const void* const* wqkv;
+    const void* const* wo;
+    const void* const* wgate;
+    const void* const* wup;
+    const void* const* wdown;
+    const void* lm_head;
+};
+
+struct TcPlan;
+
+// Build the plan (tensor maps of every weight and activation operand).  *out may be left null,
+// in which case bf16 GEMMs run on the CUDA-core kernel.
+int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, void* o, void* act, int rows_full,
+                   int rows_c, int lm_tiles_cap);
+void tc_plan_destroy(TcPlan* p);
+int tc_splits(const TcPlan* p, int wid, int m_bound);
+int tc_lm_tiles(const TcPlan* p);
+int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g, cudaStream_t s);
+
+}  // namespace focus

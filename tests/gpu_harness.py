@@ -1,0 +1,120 @@
+"""Helpers shared by the GPU tests: run the CUDA step through the C ABI, run the oracle, compare."""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+import torch
+
+import focus_synth as fs
+from oracle import focus_oracle as fo
+import parity
+
+
+def step_params(work: fs.Workload, **over) -> dict:
+    p = dict(tau=work.tau, k_min=work.k_min, k_max=work.k_max, conf_threshold=work.conf_threshold,
+             alpha=work.alpha, forced_keep_frac=work.forced_keep_frac)
+    p.update(over)
+    return p
+
+
+def limits_for(case: fs.Case, params: dict):
+    B = case.work.block
+    if params["forced_keep_frac"] >= 0:
+        mk = B
+    else:
+        mk = max(1, params["k_max"])
+    return dict(max_requests=case.work.n_requests, max_block=B, max_keep=mk,
+                max_pages_per_req=case.max_pages_per_req)
+
+
+def to_device(case: fs.Case, device="cuda:0") -> dict:
+    dev = torch.device(device)
+    m = {}
+    for k, v in case.model.items():
+        m[k] = [t.to(dev) for t in v] if isinstance(v, list) else v.to(dev)
+    return m
+
+
+def run_gpu(case: fs.Case, params: dict, model_dev: Optional[dict] = None, forced: Optional[list] = None,
+            limits: Optional[dict] = None, batch_override: Optional[dict] = None):
+    """One focused step on cuda:0 through the C ABI; returns host copies of every output and the state."""
+    from decodability_aware_token_b200 import FocusContext, StepParams
+    dev = torch.device("cuda:0")
+    model_dev = model_dev if model_dev is not None else to_device(case)
+    src = batch_override if batch_override is not None else case.batch
+    batch = {k: v.to(dev).clone() for k, v in src.items()}
+    lim = limits or limits_for(case, params)
+    sp = StepParams(**params)
+    N = batch["block_tokens"].shape[0]
+    if forced is not None:
+        idx = torch.full((N, lim["max_keep"]), -1, dtype=torch.int32)
+        cnt = torch.zeros(N, dtype=torch.int32)
+        for b, s in enumerate(forced):
+            idx[b, : len(s)] = torch.tensor(sorted(s), dtype=torch.int32)
+            cnt[b] = len(s)
+        sp.forced_keep_idx, sp.forced_keep_count = idx.to(dev), cnt.to(dev)
+    with FocusContext(case.shape, model_dev, **lim) as ctx:
+        out = ctx.step(batch, sp)
+        torch.cuda.synchronize()
+        rc, bits = ctx.device_error()
+    res = {k: (v.cpu() if v is not None else None) for k, v in out.tensors().items()}
+    res.update(block_tokens=batch["block_tokens"].cpu(), mask=batch["mask"].cpu(), ibc=batch["ibc"].cpu(),
+               device_status=rc, device_bits=bits)
+    return res
+
+
+def run_oracle(case: fs.Case, params: dict, forced=None, requests=None, max_keep=None) -> fo.OracleResult:
+    return fo.focus_step(case.shape, case.model, case.batch, tau=params["tau"], k_min=params["k_min"],
+                         k_max=params["k_max"], conf_threshold=params["conf_threshold"], alpha=params["alpha"],
+                         forced_keep_frac=params["forced_keep_frac"], forced_keep=forced, requests=requests,
+                         max_keep=max_keep)
+
+
+def subset_case(case: fs.Case, reqs) -> fs.Case:
+    batch = {k: v[reqs] if k not in ("kv_pool",) else v for k, v in case.batch.items()}
+    work = dataclasses.replace(case.work, n_requests=len(reqs))
+    return fs.Case(case.shape, work, case.model, batch, case.seed)
+
+
+def subset_gpu(gpu: dict, reqs) -> dict:
+    off = gpu["row_offsets"].numpy()
+    rows = np.concatenate([np.arange(off[b], off[b + 1]) for b in reqs]) if len(reqs) else np.zeros(0, int)
+    kc = gpu["keep_count"][reqs]
+    sub_off = torch.zeros(len(reqs) + 1, dtype=torch.int32)
+    sub_off[1:] = torch.cumsum(kc, 0)
+    return {
+        "importance": gpu["importance"][:, reqs], "keep_count": kc, "retained_idx": gpu["retained_idx"][reqs],
+        "row_offsets": sub_off, "hidden": gpu["hidden"][torch.as_tensor(rows, dtype=torch.long)],
+        "conf": gpu["conf"][reqs], "top_id": gpu["top_id"][reqs], "decoded_ids": gpu["decoded_ids"][reqs],
+        "block_tokens": gpu["block_tokens"][reqs], "mask": gpu["mask"][reqs], "ibc": gpu["ibc"][reqs],
+    }
+
+
+def check(case: fs.Case, params: dict, model_dev=None, requests=None, gpu=None, limits=None):
+    """GPU vs oracle on `case` (optionally only on sampled `requests`); re-runs with the oracle's set
+    forced if a near-tie flipped a kept set.  Returns the report dict."""
+    tol = parity.tolerance(case.shape)
+    lim = limits or limits_for(case, params)
+    if gpu is None:
+        gpu = run_gpu(case, params, model_dev, limits=lim)
+    assert gpu["device_status"] == 0, f"device error bits {gpu['device_bits']:#x}"
+    reqs = list(range(case.work.n_requests)) if requests is None else list(requests)
+    ora = run_oracle(case, params, requests=reqs, max_keep=lim["max_keep"])
+    sub = subset_case(case, reqs)
+    g = subset_gpu(gpu, reqs)
+    report, flipped = parity.compare(sub, params, ora, g, tol, sub.batch["ibc"])
+    report["flipped"] = flipped
+    if flipped:
+        kept = [ora.retained_idx[i, : ora.keep_count[i]].tolist() for i in range(len(reqs))]
+        forced_full = [[] for _ in range(case.work.n_requests)]
+        for i, b in enumerate(reqs):
+            forced_full[b] = kept[i]
+        gpu2 = run_gpu(case, params, model_dev, forced=forced_full, limits=lim)
+        assert gpu2["device_status"] == 0
+        g2 = subset_gpu(gpu2, reqs)
+        report2, fl2 = parity.compare(sub, params, ora, g2, tol, sub.batch["ibc"], check_selection=False)
+        assert not fl2
+        report["forced_rerun"] = report2
+    return report

@@ -1,0 +1,191 @@
+"""Tie-aware comparison of a GPU focused step against the CPU oracle.
+
+Rules (what is unique is compared exactly, what is not is checked for validity):
+  * importance, hidden states, confidences: max-abs error <= frac x RMS of the oracle's values
+    (frac = 2e-2 for bf16 against the float64 oracle, 1e-4 for the float32 path);
+  * kept set per request: identical wherever the oracle's delta gap at the top-k cut and its
+    |delta - tau| both exceed the selection gate; otherwise the GPU set must still be a valid top-k of
+    the oracle's deltas within that gate (and the test then re-runs the GPU with the oracle's set
+    forced to compare everything downstream);
+  * top id per kept row: identical where the oracle's top-1 logit margin exceeds the logit gate;
+    otherwise the GPU's id must be within the gate of the oracle's best logit;
+  * decoded positions / ids: identical where no threshold or fallback decision is within its gate;
+  * the intra-block KV cache: rewritten entries within tolerance, every other entry bit-identical.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+import torch
+
+from oracle import focus_oracle as fo
+
+
+@dataclasses.dataclass
+class Tol:
+    frac: float          # max-abs / RMS for importance, hidden states, confidences, cache entries
+    sel: float           # delta gate for the kept set
+    logit: float         # top-1 logit margin gate
+    conf_rel: float      # |conf - threshold| gate, relative to conf
+    log_conf: float      # fallback decision gate (log-confidence gap)
+
+
+def tolerance(shape) -> Tol:
+    if shape.dtype == "f32":
+        return Tol(frac=1e-4, sel=1e-3, logit=1e-3, conf_rel=1e-3, log_conf=1e-3)
+    # bf16 operands and activations against the float64 oracle.  A logit moves by about
+    # ||w_row|| x RMS(perturbation of the normalised hidden state); with the hidden-state tolerance
+    # of 2e-2 x RMS this bounds typical logit errors by 2e-2 x sqrt(D) x RMS(W_lm) (~1.8e-2 here).
+    return Tol(frac=2e-2, sel=1e-3, logit=None, conf_rel=4e-2, log_conf=None)
+
+
+def _np(t):
+    return t.detach().cpu().numpy() if isinstance(t, torch.Tensor) else np.asarray(t)
+
+
+def _rms(x):
+    x = np.asarray(x, dtype=np.float64)
+    return float(np.sqrt(np.mean(x * x))) if x.size else 0.0
+
+
+def close(name, got, want, frac, report):
+    got, want = np.asarray(got, np.float64), np.asarray(want, np.float64)
+    assert got.shape == want.shape, f"{name}: shape {got.shape} vs {want.shape}"
+    if got.size == 0:
+        return
+    err = float(np.max(np.abs(got - want)))
+    scale = _rms(want)
+    report[name] = (err, scale, err / scale if scale else float("inf"))
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    assert err <= frac * scale, f"{name}: max-abs error {err:.3e} > {frac} x RMS {scale:.3e}"
+
+
+def valid_selection(kept_gpu, delta, masked, params, sel_gate, B):
+    """Is `kept_gpu` a top-k of the oracle's deltas that some perturbation within the gate allows?"""
+    masked = np.asarray(masked).astype(bool)
+    tau = float(np.float32(params["tau"]))
+    f = params["forced_keep_frac"]
+    kset = set(kept_gpu)
+    if f >= 0:
+        k = min(B, fo._ceil_f32(f, B))
+        if len(kept_gpu) != k:
+            return False
+        elig = list(range(B))
+        key_grp = {j: 0 if masked[j] else 1 for j in elig}
+    else:
+        elig = [j for j in range(B) if masked[j]]
+        if not kset <= set(elig):
+            return False
+        lo = sum(1 for j in elig if delta[j] > tau + sel_gate)
+        hi = sum(1 for j in elig if delta[j] > tau - sel_gate)
+        ks = {min(min(max(fo._ceil_f32(params["alpha"], c), params["k_min"]), params["k_max"]), len(elig))
+              for c in range(lo, hi + 1)}
+        if len(kept_gpu) not in ks:
+            return False
+        key_grp = {j: 0 for j in elig}
+    out = [j for j in elig if j not in kset]
+    for a in kset:
+        for r in out:
+            if key_grp[a] > key_grp[r]:
+                return False
+            if key_grp[a] == key_grp[r] and delta[a] < delta[r] - sel_gate:
+                return False
+    return True
+
+
+def logit_of(case, hidden_row, token):
+    h = fo.rms_norm(np.asarray(hidden_row, np.float64)[None], fo._f64(case.model["final_norm"]), case.shape.rms_eps)[0]
+    return float(h @ fo._f64(case.model["lm_head"][int(token)]))
+
+
+def derived_logit_gate(case, frac):
+    w = case.model["lm_head"].float()
+    return frac * math.sqrt(case.shape.hidden) * float(w.pow(2).mean().sqrt())
+
+
+def compare(case, params: dict, ora: fo.OracleResult, gpu: dict, tol: Tol, ibc_in, check_selection=True):
+    """Assert parity; returns (report dict, list of requests whose kept set differs within the gate)."""
+    report = {}
+    N, B = ora.decoded_ids.shape
+    logit_gate = tol.logit if tol.logit is not None else derived_logit_gate(case, tol.frac)
+    lc_gate = tol.log_conf if tol.log_conf is not None else 2 * logit_gate
+    report["logit_gate"] = logit_gate
+    close("importance", gpu["importance"], ora.importance, tol.frac, report)
+    kc = _np(gpu["keep_count"])
+    ret = _np(gpu["retained_idx"])
+    masked0 = _np(case.batch["mask"]).astype(bool)
+    flipped = []
+    for b in range(N):
+        kg = ret[b, : kc[b]].tolist()
+        ko = ora.retained_idx[b, : ora.keep_count[b]].tolist()
+        assert all(x == -1 for x in ret[b, kc[b]:]), f"request {b}: padding"
+        assert kg == sorted(kg), f"request {b}: kept positions not ascending"
+        if kg == ko:
+            continue
+        exact = ora.cut_gap[b] > tol.sel and ora.tau_gap[b] > tol.sel
+        assert check_selection and not exact, (f"request {b}: kept {kg} vs oracle {ko} "
+                                               f"(cut gap {ora.cut_gap[b]:.2e}, tau gap {ora.tau_gap[b]:.2e})")
+        assert valid_selection(kg, ora.delta[b], masked0[b], params, tol.sel, B), \
+            f"request {b}: kept {kg} is not a valid top-k within the gate (oracle {ko})"
+        flipped.append(b)
+    off = _np(gpu["row_offsets"])
+    assert off[0] == 0 and np.all(np.diff(off) == kc), "row offsets are not the scan of keep counts"
+    if flipped:
+        return report, flipped
+    # downstream: identical kept sets from here on
+    close("hidden", _np(gpu["hidden"])[: off[-1]], ora.hidden, tol.frac, report)
+    conf_g, top_g = _np(gpu["conf"]), _np(gpu["top_id"])
+    mask_k = np.zeros_like(conf_g, dtype=bool)
+    for b in range(N):
+        mask_k[b, : kc[b]] = True
+    close("conf", conf_g[mask_k], ora.conf[mask_k], tol.frac, report)
+    assert np.all(conf_g[~mask_k] == 0) and np.all(top_g[~mask_k] == -1), "unused conf / top slots"
+    n_tie_ids = 0
+    for b in range(N):
+        for t in range(kc[b]):
+            if top_g[b, t] == ora.top_id[b, t]:
+                continue
+            r = off[b] + t
+            assert ora.logit_margin[b, t] <= logit_gate, (
+                f"request {b} slot {t}: top id {top_g[b, t]} vs {ora.top_id[b, t]} with margin "
+                f"{ora.logit_margin[b, t]:.3e} > gate {logit_gate:.3e}")
+            zg = logit_of(case, ora.hidden[r], top_g[b, t])
+            zo = logit_of(case, ora.hidden[r], ora.top_id[b, t])
+            assert zo - zg <= logit_gate, f"request {b} slot {t}: GPU id is {zo - zg:.3e} below the best logit"
+            n_tie_ids += 1
+    report["top_id_near_ties"] = n_tie_ids
+    dec_g = _np(gpu["decoded_ids"])
+    thr = float(np.float32(params["conf_threshold"]))
+    for b in range(N):
+        kept = ora.retained_idx[b, : ora.keep_count[b]].tolist()
+        if np.array_equal(dec_g[b], ora.decoded_ids[b]):
+            continue
+        near = (ora.thr_gap[b] <= tol.conf_rel * max(thr, 1e-30) or ora.fallback_gap[b] <= lc_gate or
+                any(ora.logit_margin[b, t] <= logit_gate for t in range(len(kept))))
+        assert near, f"request {b}: decoded {dec_g[b].tolist()} vs oracle {ora.decoded_ids[b].tolist()}"
+        # validity: decoded positions are kept masked positions, ids are the GPU's own top ids, and
+        # at least one decodes whenever a kept masked position exists
+        pos = [j for j in range(B) if dec_g[b, j] >= 0]
+        cand = [j for j in kept if masked0[b, j]]
+        assert set(pos) <= set(cand) and (len(pos) > 0) == (len(cand) > 0), f"request {b}: invalid decode set"
+        for j in pos:
+            assert dec_g[b, j] == top_g[b, kept.index(j)]
+    # tokens / mask follow the decoded ids
+    tok_g, mask_g = _np(gpu["block_tokens"]), _np(gpu["mask"])
+    tok0 = _np(case.batch["block_tokens"])
+    d = dec_g >= 0
+    assert np.array_equal(tok_g[d], dec_g[d]) and np.array_equal(tok_g[~d], tok0[~d])
+    assert np.all(mask_g[d] == 0) and np.array_equal(mask_g[~d], masked0[~d].astype(np.uint8))
+    # intra-block KV cache: written entries close, the rest untouched
+    ibc_g = gpu["ibc"].float().cpu().numpy()
+    ibc0 = ibc_in.float().cpu().numpy()
+    written = np.zeros(ibc_g.shape[:2] + (B,), dtype=bool)   # [N, L, B]
+    written[:, :2, :] = True
+    for b in range(N):
+        written[b, 2:, ora.retained_idx[b, : ora.keep_count[b]]] = True
+    w_idx = np.broadcast_to(written[:, :, None, None, :, None], ibc_g.shape)
+    close("ibc_written", ibc_g[w_idx], ora.ibc[w_idx], tol.frac, report)
+    assert np.array_equal(ibc_g[~w_idx], ibc0[~w_idx]), "an evicted position's cache entry changed"
+    return report, []

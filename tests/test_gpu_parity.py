@@ -1,0 +1,180 @@
+"""GPU parity: the CUDA focused step (through the C ABI) against the CPU oracle.
+
+Small cases span several GEMM / attention tiles and ragged tails; the full-size workloads are
+checked on sampled requests (requests are independent, so the oracle can run a subset).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import focus_synth as fs
+from gpu_harness import check, run_gpu, run_oracle, step_params, to_device, limits_for
+
+pytestmark = pytest.mark.gpu
+
+_models = {}
+
+
+def _case(name, **kw):
+    return fs.make_case(name, **kw)
+
+
+def _model(name, case):
+    if name not in _models:
+        _models.clear()
+        _models[name] = to_device(case)
+    return _models[name]
+
+
+@pytest.mark.parametrize("name", ["tiny", "small_f32", "small_bf16", "small_bf16_g4"])
+def test_adaptive_step_matches_oracle(name):
+    case = _case(name)
+    rep = check(case, step_params(case.work), _model(name, case))
+    print(name, rep)
+
+
+@pytest.mark.parametrize("name", ["tiny", "small_bf16"])
+@pytest.mark.parametrize("frac", [1.0, 0.25])
+def test_forced_fraction_matches_oracle(name, frac):
+    """Keep fraction 1 is the dense full-block step (the oracle's f = 1 is pinned to a dense forward)."""
+    case = _case(name)
+    check(case, step_params(case.work, forced_keep_frac=frac), _model(name, case))
+
+
+@pytest.mark.parametrize("name,frac,boost", [("tiny", 0.02, 60.0), ("small_bf16", 0.001, 25.0)])
+def test_confidence_threshold_path(name, frac, boost):
+    """LM-head rows of a few vocabulary entries scaled up so that some confidences clear the threshold.
+
+    The boost multiplies those logits, and with them the logit error of bf16 operands; a few rows at
+    25x keep the confidence error inside the bf16 tolerance while pushing most confidences past 0.9."""
+    case = _case(name, lm_boost_frac=frac, lm_boost=boost)
+    p = step_params(case.work)
+    gpu = run_gpu(case, p)
+    conf = gpu["conf"][gpu["conf"] > 0]
+    assert (conf > p["conf_threshold"]).any(), "the variant should exercise the threshold"
+    check(case, p, gpu=gpu)
+
+
+@pytest.mark.parametrize("name", ["small_f32", "small_bf16"])
+def test_alpha_tau_kmin_variants(name):
+    case = _case(name)
+    m = _model(name, case)
+    check(case, step_params(case.work, alpha=1.5, tau=0.002, k_min=3, k_max=case.work.k_max), m)
+    check(case, step_params(case.work, alpha=0.5, tau=-0.01, k_min=0, k_max=case.work.k_max), m)
+
+
+def _with_batch(case, **fields):
+    b = dict(case.batch)
+    b.update(fields)
+    return fs.Case(case.shape, case.work, case.model, b, case.seed)
+
+
+@pytest.mark.parametrize("name", ["tiny", "small_bf16"])
+def test_edge_no_prefix(name):
+    case = _case(name)
+    N = case.work.n_requests
+    c2 = _with_batch(case, prefix_len=torch.zeros(N, dtype=torch.int32))
+    check(c2, step_params(case.work), _model(name, case))
+
+
+@pytest.mark.parametrize("name", ["tiny", "small_bf16"])
+def test_edge_nothing_masked_keeps_nothing(name):
+    case = _case(name)
+    c2 = _with_batch(case, mask=torch.zeros_like(case.batch["mask"]))
+    gpu = run_gpu(c2, step_params(case.work), _model(name, case))
+    assert int(gpu["keep_count"].sum()) == 0 and bool((gpu["decoded_ids"] == -1).all())
+    check(c2, step_params(case.work), gpu=gpu)
+
+
+@pytest.mark.parametrize("name", ["tiny", "small_bf16"])
+def test_edge_everything_masked(name):
+    case = _case(name)
+    tok = case.batch["block_tokens"].clone()
+    tok[:] = case.shape.vocab - 1
+    c2 = _with_batch(case, mask=torch.ones_like(case.batch["mask"]), block_tokens=tok)
+    check(c2, step_params(case.work), _model(name, case))
+
+
+def test_edge_single_request_full_block_budget():
+    """N = 1, k_max = B: every masked position may be kept."""
+    case = _case("small_bf16")
+    w = dataclasses.replace(case.work, n_requests=1)
+    c2 = fs.Case(case.shape, w, case.model, {k: (v[:1] if k != "kv_pool" else v) for k, v in case.batch.items()},
+                 case.seed)
+    check(c2, step_params(w, k_max=w.block, k_min=w.block), _model("small_bf16", case))
+
+
+def test_caller_forced_set_is_honoured():
+    case = _case("small_bf16")
+    p = step_params(case.work)
+    forced = [[0, 5, 31], [], [1, 2, 3, 4, 6, 7, 8, 9], [30], [10, 20]]
+    gpu = run_gpu(case, p, _model("small_bf16", case), forced=forced)
+    for b, s in enumerate(forced):
+        assert gpu["retained_idx"][b, : gpu["keep_count"][b]].tolist() == s
+    ora = run_oracle(case, p, forced=forced, max_keep=p["k_max"])
+    import parity
+    rep, fl = parity.compare(case, p, ora, gpu, parity.tolerance(case.shape), case.batch["ibc"],
+                             check_selection=False)
+    assert not fl
+
+
+def test_bad_page_id_sets_device_error_and_does_not_fault():
+    case = _case("tiny")
+    table = case.batch["page_table"].clone()
+    table[0, 1] = 10_000                                  # no such page: the kernel skips it and flags it
+    c2 = _with_batch(case, page_table=table)
+    gpu = run_gpu(c2, step_params(case.work), _model("tiny", case))
+    from decodability_aware_token_b200 import _abi
+    assert gpu["device_status"] == _abi.FOCUS_ERR_DEVICE_BOUNDS
+    assert gpu["device_bits"] & _abi.FOCUS_DEVERR_PAGE_ID
+
+
+def test_prefix_beyond_page_table_is_clamped_and_flagged():
+    case = _case("tiny")
+    plen = case.batch["prefix_len"].clone()
+    plen[1] = 10_000
+    gpu = run_gpu(_with_batch(case, prefix_len=plen), step_params(case.work), _model("tiny", case))
+    from decodability_aware_token_b200 import _abi
+    assert gpu["device_bits"] & _abi.FOCUS_DEVERR_PREFIX
+
+
+def test_host_validation_rejects_bad_arguments():
+    from decodability_aware_token_b200 import FocusContext, StepParams, FocusError, _abi
+    case = _case("tiny")
+    m = _model("tiny", case)
+    lim = limits_for(case, step_params(case.work))
+    batch = {k: v.cuda() for k, v in case.batch.items()}
+    with FocusContext(case.shape, m, **lim) as ctx:
+        with pytest.raises(FocusError) as e:
+            ctx.step(batch, StepParams(k_min=1, k_max=case.work.block + 1))
+        assert e.value.code in (_abi.FOCUS_ERR_INVALID_ARG, _abi.FOCUS_ERR_LIMITS)
+        with pytest.raises(FocusError) as e:
+            ctx.step(batch, StepParams(k_min=1, k_max=lim["max_keep"] + 1 if lim["max_keep"] < case.work.block else 99))
+        with pytest.raises(FocusError) as e:
+            ctx.step(batch, StepParams(k_min=5, k_max=2))
+        assert e.value.code == _abi.FOCUS_ERR_INVALID_ARG
+
+
+def test_step_is_deterministic():
+    case = _case("small_bf16")
+    p = step_params(case.work)
+    m = _model("small_bf16", case)
+    a, b = run_gpu(case, p, m), run_gpu(case, p, m)
+    for k in ("importance", "keep_count", "retained_idx", "hidden", "conf", "top_id", "decoded_ids"):
+        assert torch.equal(a[k], b[k]), k
+    assert torch.equal(a["ibc"], b["ibc"])
+
+
+# ---------------------------------------------------------------- full-size workloads, sampled requests
+@pytest.mark.slow
+def test_sdar_1p7b_n32_b32_sampled():
+    case = fs.make_case("sdar1.7b_n32_b32", device="cuda:0")
+    host = fs.Case(case.shape, case.work, {k: ([t.cpu() for t in v] if isinstance(v, list) else v.cpu())
+                                           for k, v in case.model.items()},
+                   {k: v.cpu() for k, v in case.batch.items()}, case.seed)
+    p = step_params(case.work)
+    gpu = run_gpu(host, p, case.model)
+    rep = check(host, p, requests=[0, 13, 31], gpu=gpu)
+    print(rep)
