@@ -383,7 +383,8 @@ int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_l
         tw.L = L;
         tw.wqkv = c->wqkv.data(); tw.wo = c->wo.data(); tw.wgate = c->wgate.data(); tw.wup = c->wup.data();
         tw.wdown = c->wdown.data(); tw.lm_head = c->lm_head;
-        rc = tc_plan_create(&c->tc, c->dm, tw, c->h, c->o, c->act, (int)rows_full, (int)rows_c, c->lm_tiles_cap);
+        rc = tc_plan_create(&c->tc, c->dm, tw, c->h, c->o, c->act, (int)rows_full, (int)rows_c, c->lm_tiles_cap,
+                            c->err);
     }
     if (rc != FOCUS_OK) {
         cudaFree(c->ws);

@@ -21,7 +21,7 @@ struct TcPlan;
 // Build the plan (tensor maps of every weight and activation operand).  *out may be left null,
 // in which case bf16 GEMMs run on the CUDA-core kernel.
 int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, void* o, void* act, int rows_full,
-                   int rows_c, int lm_tiles_cap);
+                   int rows_c, int lm_tiles_cap, int* err);
 void tc_plan_destroy(TcPlan* p);
 int tc_splits(const TcPlan* p, int wid, int m_bound);
 int tc_lm_tiles(const TcPlan* p);

@@ -102,6 +102,18 @@ def silu(x: np.ndarray) -> np.ndarray:
     return x / (1.0 + np.exp(-x))
 
 
+def _keep(x: np.ndarray) -> np.ndarray:
+    return x
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest bfloat16 (ties to even), returned as float64."""
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+STORAGE = {"f64": _keep, "bf16": round_bf16}
+
+
 def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray):
     """Grouped-query softmax attention, no mask (block diffusion attends bidirectionally).
 
@@ -146,32 +158,37 @@ def gather_prefix(kv_pool: np.ndarray, page_row: np.ndarray, prefix_len: int, la
     return kk, vv
 
 
-def layer_forward(x, lw, shape, positions, rows, prefix_k, prefix_v, cache_k, cache_v):
+def layer_forward(x, lw, shape, positions, rows, prefix_k, prefix_v, cache_k, cache_v, store=_keep):
     """One pre-norm decoder layer on the rows `rows` (ascending block positions) of one request.
 
     cache_k / cache_v ([Hkv, B, d], float64) are the intra-block KV cache of this
     layer; the rows' fresh K/V overwrite it first (project page, Overview --
     Runtime Action: intra-block KV caching), then every row attends to the
     prefix keys plus all B cache entries.  Returns (x_out, attention probs).
+
+    `store` is applied to every activation a kernel keeps in its storage type
+    (normalised rows, q / k / v, attention output, MLP activation): the identity
+    for plain float64, or bf16 rounding to take decisions in the kernel's
+    precision.  Sums and the residual stream stay float64 either way.
     """
     hq, hkv, d = shape.n_q_heads, shape.n_kv_heads, shape.head_dim
     n = x.shape[0]
-    h = rms_norm(x, lw["attn_norm"], shape.rms_eps)
+    h = store(rms_norm(x, lw["attn_norm"], shape.rms_eps))
     qkv = h @ lw["wqkv"].T
     q = qkv[:, : hq * d].reshape(n, hq, d).transpose(1, 0, 2)
     k = qkv[:, hq * d:(hq + hkv) * d].reshape(n, hkv, d).transpose(1, 0, 2)
     v = qkv[:, (hq + hkv) * d:].reshape(n, hkv, d).transpose(1, 0, 2)
     pos = positions[rows]
-    q = rope(q, pos, shape.rope_theta)
-    k = rope(k, pos, shape.rope_theta)
+    q = store(rope(q, pos, shape.rope_theta))
+    k = store(rope(k, pos, shape.rope_theta))
     cache_k[:, rows] = k
-    cache_v[:, rows] = v
+    cache_v[:, rows] = store(v)
     keys = np.concatenate([prefix_k, cache_k], axis=1)
     vals = np.concatenate([prefix_v, cache_v], axis=1)
     o, p = attention(q, keys, vals)
-    x = x + o.transpose(1, 0, 2).reshape(n, hq * d) @ lw["wo"].T
-    h2 = rms_norm(x, lw["mlp_norm"], shape.rms_eps)
-    a = silu(h2 @ lw["wgate"].T) * (h2 @ lw["wup"].T)
+    x = x + store(o).transpose(1, 0, 2).reshape(n, hq * d) @ lw["wo"].T
+    h2 = store(rms_norm(x, lw["mlp_norm"], shape.rms_eps))
+    a = store(silu(h2 @ lw["wgate"].T) * (h2 @ lw["wup"].T))
     x = x + a @ lw["wdown"].T
     return x, p
 
@@ -237,13 +254,13 @@ def compact_rows(kept: Sequence[Sequence[int]], max_keep: int):
     return keep_count, retained, offsets, row_map
 
 
-def lm_head_conf(x: np.ndarray, final_norm: np.ndarray, lm_head: np.ndarray, eps: float):
+def lm_head_conf(x: np.ndarray, final_norm: np.ndarray, lm_head: np.ndarray, eps: float, store=_keep):
     """Final RMSNorm, logits, max-softmax confidence and top id (lowest id among equal maxima).
 
     Project page, Quality table: decoding is gated by a confidence ("Conf.").
     Returns (conf, top_id, log_conf, top-1 logit margin) per row.
     """
-    h = rms_norm(x, final_norm, eps)
+    h = store(rms_norm(x, final_norm, eps))
     z = h @ lm_head.T
     top = np.argmax(z, axis=1)               # first maximum = lowest id
     zmax = z[np.arange(z.shape[0]), top]
@@ -311,15 +328,18 @@ class OracleResult:
 def focus_step(shape, model: dict, batch: dict, *, tau: float, k_min: int, k_max: int, conf_threshold: float,
                alpha: float = 1.0, forced_keep_frac: float = -1.0, max_keep: Optional[int] = None,
                forced_keep: Optional[Sequence[Sequence[int]]] = None, requests: Optional[Sequence[int]] = None,
-               page_size: Optional[int] = None) -> OracleResult:
+               page_size: Optional[int] = None, storage: str = "f64") -> OracleResult:
     """One focused denoising step over a batch of ragged requests.
 
     shape: model shape (n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn,
     vocab, rms_eps, rope_theta); model / batch: tensors in the C ABI's layout.
     `forced_keep` replaces the selection (per request, any order) -- used to
     compare the later layers on a set chosen elsewhere.  `requests` restricts
-    the step to a subset of the batch (requests are independent).
+    the step to a subset of the batch (requests are independent).  `storage`
+    "bf16" rounds activations where a bf16 kernel stores them (see
+    layer_forward), so that decisions are taken in the kernel's precision.
     """
+    store = STORAGE[storage]
     tokens = _i64(batch["block_tokens"])
     mask = _i64(batch["mask"]).astype(bool)
     prefix_len = _i64(batch["prefix_len"])
@@ -356,7 +376,8 @@ def focus_step(shape, model: dict, batch: dict, *, tau: float, k_min: int, k_max
         lw = layer_weights(l)
         for b in range(N):
             pk, pv = gather_prefix(kv_pool, table[b], int(prefix_len[b]), l, S)
-            x[b], p = layer_forward(x[b], lw, shape, positions[b], all_rows, pk, pv, ibc[b, l, 0], ibc[b, l, 1])
+            x[b], p = layer_forward(x[b], lw, shape, positions[b], all_rows, pk, pv, ibc[b, l, 0], ibc[b, l, 1],
+                                    store)
             importance[l, b] = importance_from_probs(p, int(prefix_len[b]))
     delta = importance[1] - importance[0]
 
@@ -383,7 +404,7 @@ def focus_step(shape, model: dict, batch: dict, *, tau: float, k_min: int, k_max
                 continue
             pk, pv = gather_prefix(kv_pool, table[b], int(prefix_len[b]), l, S)
             xc[b], _ = layer_forward(xc[b], lw, shape, positions[b], np.asarray(kept[b]), pk, pv,
-                                     ibc[b, l, 0], ibc[b, l, 1])
+                                     ibc[b, l, 0], ibc[b, l, 1], store)
 
     # LM head, confidence, decode
     final_norm, lm_head = _f64(model["final_norm"]), _f64(model["lm_head"])
@@ -398,7 +419,7 @@ def focus_step(shape, model: dict, batch: dict, *, tau: float, k_min: int, k_max
         k = len(kept[b])
         if k == 0:
             continue
-        c, t, lc, mg = lm_head_conf(xc[b], final_norm, lm_head, shape.rms_eps)
+        c, t, lc, mg = lm_head_conf(xc[b], final_norm, lm_head, shape.rms_eps, store)
         conf[b, :k], top_id[b, :k], log_conf[b, :k], margin[b, :k] = c, t, lc, mg
         dec, thr_gap[b], fb_gap[b] = threshold_decode(kept[b], mask[b], c, t, conf_threshold)
         for j, tok in dec.items():

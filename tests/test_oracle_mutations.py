@@ -68,7 +68,7 @@ def _select_high_index_on_ties(delta, masked, *, tau, k_min, k_max, alpha=1.0, f
 
 
 def _layer_variant(write_cache_first=True, mlp_residual=True):
-    def layer(x, lw, shape, positions, rows, prefix_k, prefix_v, cache_k, cache_v):
+    def layer(x, lw, shape, positions, rows, prefix_k, prefix_v, cache_k, cache_v, store=fo._keep):
         hq, hkv, d = shape.n_q_heads, shape.n_kv_heads, shape.head_dim
         n = x.shape[0]
         h = fo.rms_norm(x, lw["attn_norm"], shape.rms_eps)
@@ -93,8 +93,8 @@ def _layer_variant(write_cache_first=True, mlp_residual=True):
     return layer
 
 
-def _lm_head_highest_id(x, g, w, eps):
-    conf, top, lc, mg = _orig["lm_head_conf"](x, g, w, eps)
+def _lm_head_highest_id(x, g, w, eps, store=fo._keep):
+    conf, top, lc, mg = _orig["lm_head_conf"](x, g, w, eps, store)
     z = fo.rms_norm(x, g, eps) @ w.T
     return conf, z.shape[1] - 1 - np.argmax(z[:, ::-1], axis=1), lc, mg          # slip: highest id on ties
 

@@ -123,6 +123,31 @@ def test_silu_identities():
     assert abs(fo.silu(np.array([40.0]))[0] - 40.0) < 1e-12
 
 
+def test_bf16_storage_rounding_closed_forms():
+    """bf16 keeps 8 significant bits: 1 + 2^-8 is a tie (to even: 1), just above it rounds up to 1 + 2^-7."""
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 2 ** -8 + 2 ** -20, 1.0 + 3 * 2 ** -8, -3.0 - 2 ** -7, 2.0 ** -130])
+    want = np.array([1.0, 1.0, 1.0 + 2 ** -7, 1.0 + 2 ** -6, -3.0, 2.0 ** -130])
+    np.testing.assert_array_equal(fo.round_bf16(x), want)
+    y = rng.normal(size=1000) * 10
+    r = fo.round_bf16(y)
+    assert np.all(np.abs(r - y) <= np.abs(y) * 2.0 ** -8)        # half an ulp of an 8-bit significand
+    np.testing.assert_array_equal(fo.round_bf16(r), r)             # idempotent
+
+
+def test_bf16_storage_only_rounds_activations():
+    """storage='f64' is the plain step; storage='bf16' moves hidden states by about the bf16 ulp."""
+    case = fs.make_case("tiny")
+    w = case.work
+    kw = dict(tau=w.tau, k_min=w.k_min, k_max=w.k_max, conf_threshold=w.conf_threshold, forced_keep_frac=1.0)
+    a = fo.focus_step(case.shape, case.model, case.batch, **kw)
+    b = fo.focus_step(case.shape, case.model, case.batch, storage="f64", **kw)
+    c = fo.focus_step(case.shape, case.model, case.batch, storage="bf16", **kw)
+    np.testing.assert_array_equal(a.hidden, b.hidden)
+    rel = np.abs(c.hidden - a.hidden).max() / np.sqrt(np.mean(a.hidden ** 2))
+    assert 1e-5 < rel < 2e-2
+    assert np.all(fo.round_bf16(c.ibc) == c.ibc)                   # the cache holds bf16 values
+
+
 # ---------------------------------------------------------------- selection / compaction
 def test_select_golden_cases():
     data = json.load(open(os.path.join(GOLDEN, "select_cases.json")))
