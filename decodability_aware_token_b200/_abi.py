@@ -24,7 +24,8 @@ FOCUS_DTYPE_BF16 = 1
 
 # every symbol include/focus.h declares (checked by the CPU tests)
 EXPORTED = ("focus_init", "focus_step", "focus_destroy", "focus_status_string", "focus_get_device_error",
-            "focus_workspace_bytes", "focus_last_step_launches", "focus_profile_begin", "focus_profile_end")
+            "focus_workspace_bytes", "focus_last_step_launches", "focus_profile_begin", "focus_profile_end",
+            "focus_lm_head_conf_noalloc")
 
 KERNEL_CLASSES = ("embed_norm", "qkv_finalize", "attn_score", "attn_ragged", "row_norm", "select", "decode",
                   "gemm_full_qkv", "gemm_full_o", "gemm_full_gateup", "gemm_full_down",
@@ -96,5 +97,8 @@ def load():
     lib.focus_profile_begin.restype = C.c_int
     lib.focus_profile_end.argtypes = [C.c_void_p, C.POINTER(C.c_float), C.POINTER(C.c_int32)]
     lib.focus_profile_end.restype = C.c_int
+    lib.focus_lm_head_conf_noalloc.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_int32,
+                                               C.c_float, C.c_void_p, C.c_void_p, C.c_void_p]
+    lib.focus_lm_head_conf_noalloc.restype = C.c_int
     _lib = lib
     return lib

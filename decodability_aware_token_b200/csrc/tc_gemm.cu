@@ -11,352 +11,18 @@
 // epilogue.  Operand tiles are K-major with the 128-byte swizzle that TMA writes; no cluster multicast.
 // Every mbarrier wait is bounded: on expiry the kernel flags FOCUS_DEVERR_TIMEOUT, still waits (bounded)
 // for its own in-flight copies, frees its TMEM and returns.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include <math_constants.h>
-
 #include <unordered_map>
 
 #include "tc_gemm.h"
+#include "tc_gemm_kernel.cuh"
 
 namespace focus {
 
 namespace {
 
-constexpr int BK = 64;                     // K elements per stage (128 bytes of bf16: one swizzle row)
-constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Wait for the phase with `parity` to complete; false (and the timeout bit) if it does not in ~1 s.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
-    const uint32_t a = smem_u32(bar);
-    if (mbar_try(a, parity)) return true;
-    const long long t0 = clock64();
-    while (!mbar_try(a, parity)) {
-        if (clock64() - t0 > kWaitCycles) {
-            raise_err(err, FOCUS_DEVERR_TIMEOUT);
-            return false;
-        }
-    }
-    return true;
-}
-
-__device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Shared-memory matrix descriptor: K-major tile written by TMA with the 128-byte swizzle;
-// 8-row core groups 1024 bytes apart (stride byte offset), leading byte offset unused for this layout.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3FFF);        // start address
-    d |= (uint64_t)1 << 16;                       // leading byte offset (16 B, unused)
-    d |= (uint64_t)(1024 >> 4) << 32;             // stride byte offset
-    d |= (uint64_t)1 << 46;                       // descriptor version for tcgen05
-    d |= (uint64_t)2 << 61;                       // 128-byte swizzle
-    return d;
-}
-
-// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator, both K-major, M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
-    return (1u << 4)                    // D format: f32
-           | (1u << 7)                  // A format: bf16
-           | (1u << 10)                 // B format: bf16
-           | ((uint32_t)(N >> 3) << 17) // N / 8
-           | ((uint32_t)(M >> 4) << 24);// M / 16
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
-        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
-// 32 consecutive fp32 columns of this warp's 32 TMEM lanes (one row per thread).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-template <int BN, int MSUB, int STAGES>
-struct TcShape {
-    static constexpr int BM = 128 * MSUB;
-    static constexpr int A_BYTES = BM * BK * 2;
-    static constexpr int B_BYTES = BN * BK * 2;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;  // + alignment slack
-    static constexpr int TMEM_COLS = (MSUB * BN <= 32) ? 32 : (MSUB * BN <= 64) ? 64 : (MSUB * BN <= 128) ? 128
-                                     : (MSUB * BN <= 256) ? 256 : 512;
-    static_assert(MSUB * BN <= 512, "accumulators exceed TMEM");
-    static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "tcgen05 N for M = 128");
-};
-
-template <int BN, int MSUB, int STAGES, int EPI>
-__global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                                                         const __grid_constant__ CUtensorMap tmB,
-                                                         const __grid_constant__ CUtensorMap tmB2, GemmArgs g,
-                                                         int* err) {
-    using S = TcShape<BN, MSUB, STAGES>;
-    extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full_bar[STAGES];
-    __shared__ __align__(8) uint64_t empty_bar[STAGES];
-    __shared__ __align__(8) uint64_t accum_bar;
-    __shared__ uint32_t tmem_slot;
-
-    const int M = g.M_dev ? *g.M_dev : g.M_bound;
-    const int m0 = blockIdx.y * S::BM;
-    if (m0 >= M) return;  // whole CTA, before any barrier or TMEM use
-    const int n_tile = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-    // K blocks of this split
-    const int nk_all = g.K / BK;
-    const int split = blockIdx.z, splits = gridDim.z;
-    const int kb0 = (int)((long long)nk_all * split / splits);
-    const int kb1 = (int)((long long)nk_all * (split + 1) / splits);
-    const int nk = kb1 - kb0;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], 1);
-        }
-        mbar_init(&accum_bar, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
-                     "r"((uint32_t)S::TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = tmem_slot;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            // ---- TMA producer
-            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
-            if (EPI == EPI_SWIGLU) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB2) : "memory");
-            int issued = 0;
-            for (int i = 0; i < nk; ++i) {
-                const int s = i % STAGES;
-                const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-                if (!mbar_wait(&empty_bar[s], ph ^ 1u, err)) break;
-                uint8_t* a_dst = smem + s * S::STAGE_BYTES;
-                uint8_t* b_dst = a_dst + S::A_BYTES;
-                mbar_expect_tx(&full_bar[s], S::STAGE_BYTES);
-                const int kx = (kb0 + i) * BK;
-                tma_load_2d(&tmA, &full_bar[s], a_dst, kx, m0);
-                if (EPI == EPI_SWIGLU) {
-                    tma_load_2d(&tmB, &full_bar[s], b_dst, kx, n_tile * (BN / 2));
-                    tma_load_2d(&tmB2, &full_bar[s], b_dst + (BN / 2) * BK * 2, kx, n_tile * (BN / 2));
-                } else {
-                    tma_load_2d(&tmB, &full_bar[s], b_dst, kx, n_tile * BN);
-                }
-                ++issued;
-            }
-            // never leave with copies in flight: wait (bounded) for the last stages issued
-            for (int i = issued - 1; i >= 0 && i >= issued - STAGES; --i)
-                mbar_wait(&full_bar[i % STAGES], (uint32_t)(i / STAGES) & 1u, err);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        if (lane == 0) {
-            // ---- MMA issuer (one thread)
-            constexpr uint32_t idesc = idesc_bf16(128, BN);
-            for (int i = 0; i < nk; ++i) {
-                const int s = i % STAGES;
-                const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-                if (!mbar_wait(&full_bar[s], ph, err)) break;
-                tc_fence_after();
-                const uint32_t a_addr = smem_u32(smem + s * S::STAGE_BYTES);
-                const uint32_t b_addr = a_addr + S::A_BYTES;
-#pragma unroll
-                for (int ms = 0; ms < MSUB; ++ms) {
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t ad = smem_desc_sw128(a_addr + ms * 128 * 128 + kk * 32);
-                        const uint64_t bd = smem_desc_sw128(b_addr + kk * 32);
-                        mma_bf16(tmem + ms * BN, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-                    }
-                }
-                mma_commit(&empty_bar[s]);  // slot free once these MMAs have read it
-            }
-            mma_commit(&accum_bar);         // accumulators complete
-        }
-        __syncwarp();
-    } else {
-        // ---- epilogue: warps 2..5, TMEM lane quarter = warp % 4
-        const int quarter = warp & 3;
-        const bool ok = mbar_wait(&accum_bar, 0, err);
-        tc_fence_after();
-#pragma unroll 1
-        for (int ms = 0; ms < MSUB; ++ms) {
-            const int row = m0 + ms * 128 + quarter * 32 + lane;
-            const bool live = ok && row < M && nk > 0;
-            const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + ms * BN;
-            if (EPI == EPI_PARTIAL) {
-                float* out = g.part + (size_t)split * g.split_stride + (size_t)row * g.N + (size_t)n_tile * BN;
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    float v[32];
-                    tmem_ld32(tbase + c0, v);
-                    if (live) {
-                        float4* o4 = reinterpret_cast<float4*>(out + c0);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) o4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                    }
-                }
-            } else if (EPI == EPI_SWIGLU) {
-                bf16* out = reinterpret_cast<bf16*>(g.act) + (size_t)row * g.N + (size_t)n_tile * (BN / 2);
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN / 2; c0 += 32) {
-                    float gt[32], up[32];
-                    tmem_ld32(tbase + c0, gt);
-                    tmem_ld32(tbase + BN / 2 + c0, up);
-                    if (live) {
-                        uint4* o4 = reinterpret_cast<uint4*>(out + c0);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int i0 = 8 * q + 2 * e;
-                                const float a0 = gt[i0] / (1.f + expf(-gt[i0])) * up[i0];
-                                const float a1 = gt[i0 + 1] / (1.f + expf(-gt[i0 + 1])) * up[i0 + 1];
-                                __nv_bfloat162 p2 = __floats2bfloat162_rn(a0, a1);
-                                w[e] = *reinterpret_cast<uint32_t*>(&p2);
-                            }
-                            o4[q] = make_uint4(w[0], w[1], w[2], w[3]);
-                        }
-                    }
-                }
-            } else {
-                // vocabulary tile statistics of this row, online over 32-column chunks
-                float mx = -CUDART_INF_F, se = 0.f;
-                int arg = 0x7fffffff;
-                const int col0 = n_tile * BN;
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    float v[32];
-                    tmem_ld32(tbase + c0, v);
-                    float cm = -CUDART_INF_F;
-                    int ca = 0x7fffffff;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const bool in = col0 + c0 + i < g.N;
-                        if (in && v[i] > cm) {
-                            cm = v[i];
-                            ca = col0 + c0 + i;
-                        }
-                    }
-                    // (no early exit: every lane must reach the next tcgen05.ld)
-                    if (cm > mx) {
-                        se = (mx == -CUDART_INF_F) ? 0.f : se * expf(mx - cm);
-                        mx = cm;
-                        arg = ca;
-                    }
-                    if (cm != -CUDART_INF_F) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (col0 + c0 + i < g.N) se += expf(v[i] - mx);
-                    }
-                }
-                if (live) {
-                    const size_t idx = (size_t)row * g.n_tiles + n_tile;
-                    g.lm_max[idx] = mx;
-                    g.lm_sum[idx] = se;
-                    g.lm_arg[idx] = arg;
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 1) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)S::TMEM_COLS)
-                     : "memory");
-    }
-}
+using namespace tc;
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-// 2-D bf16 row-major [rows, cols] tensor, box = [box_rows, 64 cols], 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 constexpr int kBN = 128, kMSUB = 2, kStages = 4;
 using Shape = TcShape<kBN, kMSUB, kStages>;
 
