@@ -82,6 +82,11 @@ bool lim_ok(const focus_limits* l) {
 
 int lm_tiles(const focus_model_cfg* c) { return (c->vocab + kSimtTileN - 1) / kSimtTileN; }
 
+// query tiles per (request, KV head) of the full-block attention (bf16 tensor-core kernel), 1 otherwise
+int imp_tiles(const focus_model_cfg* c, const focus_limits* l) {
+    return c->dtype == FOCUS_DTYPE_BF16 ? attention_q_tiles(l->max_block, c->n_q_heads / c->n_kv_heads) : 1;
+}
+
 Layout plan(const focus_model_cfg* c, const focus_limits* l) {
     const size_t elt = c->dtype == FOCUS_DTYPE_BF16 ? 2 : 4;
     const size_t rows_full = (size_t)l->max_requests * l->max_block;
@@ -98,7 +103,7 @@ Layout plan(const focus_model_cfg* c, const focus_limits* l) {
         rows_full * HD * elt,                               // 4 o
         rows_full * F * elt,                                // 5 act
         part_rows * widest * 4,                             // 6 part
-        2 * (size_t)l->max_requests * c->n_kv_heads * l->max_block * 4,  // 7 imp_part
+        2 * (size_t)l->max_requests * c->n_kv_heads * imp_tiles(c, l) * l->max_block * 4,  // 7 imp_part
         rows_c * 4, rows_c * 4, rows_c * 4,                 // 8-10 row_req, row_pos, row_src
         64,                                                 // 11 n_rows
         rows_c * lm_tiles(c) * 4,                           // 12 lm_max
@@ -146,6 +151,13 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
     T* ibc = reinterpret_cast<T*>(in->ibc);
     auto W = [](const void* ptr) { return reinterpret_cast<const T*>(ptr); };
     const bool tc = c->cfg.dtype == FOCUS_DTYPE_BF16 && c->tc != nullptr;
+    const bool bf = c->cfg.dtype == FOCUS_DTYPE_BF16;
+    const int G = dm.Hq / dm.Hkv;
+    const int qt_full = bf ? attention_q_tiles(B, G) : 1;         // importance partial groups per KV head
+    const int qt_kept = bf ? attention_q_tiles(k_cap, G) : 1;
+    auto attention = [&](const AttnArgs& args, int q_tiles) {
+        return bf ? launch_attention_tc(args, q_tiles, s) : launch_attention<T>(args, s);
+    };
 
     // every launch goes through here: launch accounting and optional per-class event timing
     int launches = 0;
@@ -194,8 +206,8 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
         });
         at.layer = l;
         at.row_offsets = nullptr;
-        at.imp_part = c->imp_part + (size_t)l * N * dm.Hkv * B;
-        run(FOCUS_K_ATTN_SCORE, [&] { return launch_attention<T>(at, s); });
+        at.imp_part = c->imp_part + (size_t)l * N * dm.Hkv * qt_full * B;
+        run(FOCUS_K_ATTN_SCORE, [&] { return attention(at, qt_full); });
         gemm(FOCUS_K_GEMM_FULL_O, EPI_PARTIAL, c->o, c->wo[l], nullptr, rows_full, nullptr, dm.D, dm.Hq * dm.d, 1, W_O,
              nullptr);
         run(FOCUS_K_ROW_NORM, [&] {
@@ -214,7 +226,8 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
     }
     // ---- delta, budget, top-k, row map
     SelectArgs sa{};
-    sa.imp_part = c->imp_part; sa.mask = in->mask; sa.N = N; sa.B = B; sa.Hkv = dm.Hkv; sa.max_keep = c->lim.max_keep;
+    sa.imp_part = c->imp_part; sa.mask = in->mask; sa.N = N; sa.B = B; sa.groups = dm.Hkv * qt_full;
+    sa.max_keep = c->lim.max_keep;
     sa.tau = p->tau; sa.alpha = p->alpha; sa.forced_frac = p->forced_keep_frac; sa.k_min = p->k_min; sa.k_max = p->k_max;
     sa.forced_idx = p->forced_keep_idx; sa.forced_cnt = p->forced_keep_count;
     sa.keep_count = out->keep_count; sa.retained_idx = out->retained_idx; sa.row_offsets = out->row_offsets;
@@ -241,7 +254,7 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
         at.layer = l;
         at.row_offsets = out->row_offsets;
         at.imp_part = nullptr;
-        run(FOCUS_K_ATTN_RAGGED, [&] { return launch_attention<T>(at, s); });
+        run(FOCUS_K_ATTN_RAGGED, [&] { return attention(at, qt_kept); });
         gemm(FOCUS_K_GEMM_O, EPI_PARTIAL, c->o, c->wo[l], nullptr, R_bound, c->n_rows, dm.D, dm.Hq * dm.d, sp_o, W_O,
              nullptr);
         run(FOCUS_K_ROW_NORM, [&] {

@@ -47,12 +47,16 @@ struct AttnArgs {
     int* err;
 };
 template <typename T> int launch_attention(const AttnArgs& a, cudaStream_t s);
+// bf16, head_dim 128: tensor-core kernel (attention_tc.cu); the full phase writes its importance column
+// sums per (KV head, 64-vector query tile): imp_part [N, Hkv, q_tiles, B]
+int launch_attention_tc(const AttnArgs& a, int q_tiles, cudaStream_t s);
+int attention_q_tiles(int B, int G);
 
 // ---- selection + compaction metadata (select.cu) ------------------------------
 struct SelectArgs {
-    const float* imp_part;      // [2, N, Hkv, B]
+    const float* imp_part;      // [2, N, groups, B]: per-group importance partials, summed in group order
     const uint8_t* mask;        // [N, B]
-    int N, B, Hkv, max_keep;
+    int N, B, groups, max_keep;
     float tau, alpha, forced_frac;
     int k_min, k_max;
     const int32_t* forced_idx;  // optional [N, max_keep]

@@ -32,7 +32,7 @@ __global__ void __launch_bounds__(1024) select_kernel(SelectArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int B = a.B;
     const bool forced = a.forced_frac >= 0.f;
-    const size_t layer_stride = (size_t)a.N * a.Hkv * B;
+    const size_t layer_stride = (size_t)a.N * a.groups * B;
 
     for (int b = warp; b < a.N; b += nw) {
         float dl[2];
@@ -44,9 +44,9 @@ __global__ void __launch_bounds__(1024) select_kernel(SelectArgs a) {
             msk[h] = false;
             if (valid[h]) {
                 float i0 = 0.f, i1 = 0.f;
-                for (int g = 0; g < a.Hkv; ++g) {  // KV groups in order: deterministic
-                    i0 += a.imp_part[((size_t)b * a.Hkv + g) * B + j];
-                    i1 += a.imp_part[layer_stride + ((size_t)b * a.Hkv + g) * B + j];
+                for (int g = 0; g < a.groups; ++g) {  // partial groups in order: deterministic
+                    i0 += a.imp_part[((size_t)b * a.groups + g) * B + j];
+                    i1 += a.imp_part[layer_stride + ((size_t)b * a.groups + g) * B + j];
                 }
                 dl[h] = i1 - i0;
                 msk[h] = a.mask[(size_t)b * B + j] != 0;
