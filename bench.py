@@ -16,6 +16,7 @@ one request of the same workload per step.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -51,7 +52,21 @@ def parse():
     ap.add_argument("--cpu-baseline-requests", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager focus_step calls instead of graph replays")
+    ap.add_argument("--layers", type=int, default=None, help="override the layer count (profiling cases)")
+    ap.add_argument("--requests", type=int, default=None, help="override the request count (profiling cases)")
     return ap.parse_args()
+
+
+def make_workload(args, seed, device):
+    """The named workload, optionally with fewer layers / other request counts for small profiling cases."""
+    sname, wname = fs.CASES[args.workload]
+    shape, work = fs.MODEL_SHAPES[sname], fs.WORKLOADS[wname]
+    if args.layers is not None:
+        shape = dataclasses.replace(shape, n_layers=args.layers)
+    if args.requests is not None:
+        work = dataclasses.replace(work, n_requests=args.requests)
+    return fs.make_case(args.workload, seed=seed, device=device, shape=shape, work=work)
 
 
 def workload_desc(case: fs.Case) -> str:
@@ -202,7 +217,7 @@ def blas_threads():
 
 def run_reference(args):
     """The oracle on the host cores: each step is one request of the workload (requests cycle)."""
-    case = fs.make_case(args.workload)
+    case = make_workload(args, fs.SEEDS.get(args.workload, 1234), "cpu")
     model64 = {k: ([t.to(torch.float64).numpy() for t in v] if isinstance(v, list) else v.to(torch.float64).numpy())
                for k, v in case.model.items()}
     N = case.work.n_requests
@@ -249,7 +264,7 @@ def main():
             dist.barrier()
 
     base = fs.SEEDS.get(args.workload, 1234)
-    case = fs.make_case(args.workload, seed=base + 7919 * rank, device=dev)    # this rank's requests
+    case = make_workload(args, base + 7919 * rank, dev)    # this rank's requests
     w, shp = case.work, case.shape
     N, B = w.n_requests, w.block
     params = StepParams(w.tau, w.k_min, w.k_max, w.conf_threshold, w.alpha, w.forced_keep_frac)
@@ -259,63 +274,98 @@ def main():
     K, Wm = args.steps, max(3, args.warmup)
     tok0, mask0, ibc0 = case.batch["block_tokens"], case.batch["mask"], case.batch["ibc"]
 
-    def fresh_state():
-        b = dict(case.batch)
-        b["block_tokens"], b["mask"], b["ibc"] = tok0.clone(), mask0.clone(), ibc0.clone()
-        return b
-
-    # every step gets the workload's initial state (a step decodes in place, which would shrink later steps)
-    states = [fresh_state() for _ in range(Wm + K)]
-    outs = [StepOutputs.alloc(N, B, mk, shp.hidden, dev, importance=False, hidden=False) for _ in range(Wm + K)]
+    # The step decodes in place: every timed step starts from the workload's initial tokens and mask
+    # (two small copies).  The intra-block KV cache needs no reset: a step rewrites every entry it reads
+    # before reading it (all positions at layers 0-1, the kept rows at later layers), so after one step
+    # it is a fixed point and each step repeats the same work.
+    st = dict(case.batch)
+    st["block_tokens"], st["mask"], st["ibc"] = tok0.clone(), mask0.clone(), ibc0.clone()
+    out = StepOutputs.alloc(N, B, mk, shp.hidden, dev, importance=False, hidden=False)
     stream = torch.cuda.current_stream(dev)
 
+    def one_step():
+        st["block_tokens"].copy_(tok0)
+        st["mask"].copy_(mask0)
+        ctx.step(st, params, out)
+
     for i in range(Wm):
-        ctx.step(states[i], params, outs[i])
+        one_step()
     torch.cuda.synchronize(dev)
     launches_per_step = ctx.last_step_launches()
-    kept = outs[0].keep_count.cpu()
+    kept = out.keep_count.cpu()
     R = int(kept.sum())
     plen = case.batch["prefix_len"].cpu()
 
-    # which kernel class dominates (a few untimed steps per class, then fresh states again)
+    # device time per kernel class (untimed: one captured step per class, event pairs around its launches)
     from decodability_aware_token_b200 import _abi
     per_class = {}
     if args.roofline_kernel == "auto":
-        probe = fresh_state()
         for kc in _abi.KERNEL_CLASSES:
             ctx.profile_begin(kc, 4096)
-            for _ in range(2):
-                probe["block_tokens"].copy_(tok0); probe["mask"].copy_(mask0); probe["ibc"].copy_(ibc0)
-                ctx.step(probe, params, outs[0])
-            ms, n = ctx.profile_end()
-            per_class[kc] = (ms / 2.0, n / 2.0)
+            try:
+                if args.eager:
+                    one_step()
+                else:
+                    probe = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(probe):
+                        one_step()
+                    probe.replay()
+                    torch.cuda.synchronize(dev)
+                ms, n = ctx.profile_end()
+            except RuntimeError:
+                ms, n = 0.0, 0
+            per_class[kc] = (ms, n)
         roof_class = max(per_class, key=lambda k: per_class[k][0])
-        del probe
     else:
         roof_class = args.roofline_kernel
     torch.cuda.synchronize(dev)
+
+    # the step is captured once as a CUDA graph (its launch sequence depends only on host-visible sizes),
+    # with event pairs around every launch of the roofline kernel class; each replay runs one step
+    graph = None
+    if not args.eager:
+        ctx.profile_begin(roof_class, 4096)
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                one_step()
+            graph.replay()
+            torch.cuda.synchronize(dev)
+        except RuntimeError as exc:  # capture refused: time eager calls instead, and say so
+            print(f"CUDA graph capture failed ({exc}); timing eager calls", file=sys.stderr)
+            graph = None
+            args.eager = True
+            ctx.profile_end()
 
     # ---- timed region: device events on the launching stream, max over ranks
     sampler = ClockSampler(local)
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize(dev)
-    ctx.profile_begin(roof_class, max(1, K * 64))
+    if args.eager:
+        ctx.profile_begin(roof_class, max(1, K * 64))
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     tw0 = time.time()
     ev0.record(stream)
     for i in range(K):
-        ctx.step(states[Wm + i], params, outs[Wm + i])
+        if graph is not None:
+            graph.replay()
+        else:
+            one_step()
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     tw1 = time.time()
-    kern_ms, kern_n = ctx.profile_end()
+    try:
+        kern_ms, kern_n = ctx.profile_end()   # graph: the event pairs of the last replay
+    except RuntimeError as exc:
+        print(f"kernel timing unavailable ({exc})", file=sys.stderr)
+        kern_ms, kern_n = 0.0, 0
     barrier()
     time.sleep(0.1)
     sampler.stop()
     clocks = sampler.summary(tw0, tw1)
     elapsed = ev0.elapsed_time(ev1)
-    decoded = sum(int((o.decoded_ids >= 0).sum()) for o in outs[Wm:])
+    decoded = int((out.decoded_ids >= 0).sum()) * K     # every step repeats the same (deterministic) work
     t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
     tk = torch.tensor([decoded], dtype=torch.float64, device=dev)
     if world > 1:
@@ -323,35 +373,31 @@ def main():
         dist.all_reduce(tk, op=dist.ReduceOp.SUM)
     max_ms, total_decoded = float(t.item()), float(tk.item())
     value = total_decoded / (max_ms / 1e3)
+    del graph
 
-    # ---- end to end through the public API with pinned host buffers
+    # ---- end to end through the public API (eager calls) with pinned host buffers
     e2e = None
     if not args.no_e2e:
         host_in = {k: case.batch[k].cpu().pin_memory() for k in ("block_tokens", "mask", "prefix_len", "page_table")}
-        host_in["block_tokens"].copy_(tok0.cpu())
-        host_in["mask"].copy_(mask0.cpu())
-        for st in states:
-            st["ibc"].copy_(ibc0)
-        outs_h = [StepOutputs.alloc(N, B, mk, shp.hidden, "cpu", importance=False, hidden=False, pin_memory=True)
-                  for _ in range(K)]
+        out_h = StepOutputs.alloc(N, B, mk, shp.hidden, "cpu", importance=False, hidden=False, pin_memory=True)
+        names = ("keep_count", "retained_idx", "decoded_ids", "conf", "top_id")
         h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-        d2h = sum(getattr(outs_h[0], k).numel() * getattr(outs_h[0], k).element_size()
-                  for k in ("keep_count", "retained_idx", "decoded_ids", "conf", "top_id"))
+        d2h = sum(getattr(out_h, k).numel() * getattr(out_h, k).element_size() for k in names)
         torch.cuda.synchronize(dev)
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_dec = 0
         e0.record(stream)
         for i in range(K):
-            st = states[Wm + i]
             for k_, v in host_in.items():
                 st[k_].copy_(v, non_blocking=True)
-            o = ctx.step(st, params, outs[Wm + i])
-            for k_ in ("keep_count", "retained_idx", "decoded_ids", "conf", "top_id"):
-                getattr(outs_h[i], k_).copy_(getattr(o, k_), non_blocking=True)
+            o = ctx.step(st, params, out)
+            for k_ in names:
+                getattr(out_h, k_).copy_(getattr(o, k_), non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = e0.elapsed_time(e1)
-        e_dec = sum(int((o.decoded_ids >= 0).sum()) for o in outs_h)
+        e_dec = int((out_h.decoded_ids >= 0).sum()) * K
         te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
         tke = torch.tensor([e_dec], dtype=torch.float64, device=dev)
         if world > 1:
@@ -388,6 +434,7 @@ def main():
                                 for k, v in case.model.items()},
                        {k: v.cpu() for k, v in case.batch.items()}, case.seed)
         host.batch["block_tokens"], host.batch["mask"], host.batch["ibc"] = tok0.cpu(), mask0.cpu(), ibc0.cpu()
+        del st
         nreq = min(N, args.cpu_baseline_requests)
         ctok, csec = oracle_tokens_per_s(host, range(nreq))
         cpu = {"value": ctok / csec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
@@ -399,9 +446,13 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm,
             "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if shp.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": {"workload": args.workload, "desc": workload_desc(case), "requests_per_gpu": N,
+            "config": {"workload": args.workload + ("" if args.layers is None and args.requests is None else
+                                                    f" (layers={shp.n_layers}, requests={N})"),
+                       "desc": workload_desc(case), "requests_per_gpu": N,
                        "global_batch": N * world, "block": B, "kept_rows_per_step": R,
                        "decoded_per_step": total_decoded / K / world,
+                       "launch": "eager focus_step calls" if args.eager else
+                                 "CUDA graph of one focus_step, one replay per step (tokens/mask restored by two copies)",
                        "l2": "inputs larger than L2 (3.4 GB of weights and ~2.4 GB of KV pages streamed per step)",
                        "parallelism": f"replicas x{world} (requests sharded, no collective)"},
             "gpu_launches": launches_per_step * K,

@@ -123,6 +123,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attention_simt_kernel(AttnArg
 
 }  // namespace
 
+bool configure_attention_kernels() {
+    return max_shared_carveout((const void*)attention_simt_kernel<float>) &&
+           max_shared_carveout((const void*)attention_simt_kernel<bf16>) && configure_attention_tc_kernels();
+}
+
 template <typename T>
 int launch_attention(const AttnArgs& a, cudaStream_t s) {
     if (a.N <= 0) return 0;

@@ -23,29 +23,32 @@
 #include <math_constants.h>
 
 #include "launch.h"
+#include "tc_gemm_kernel.cuh"
 
 namespace focus {
 
 namespace {
 
+using tc::mbar_expect_tx;
+using tc::mbar_init;
+using tc::mbar_wait;
+using tc::tma_load_2d;
+
 constexpr int kChunk = 64;      // keys per chunk
 constexpr int kD = 128;         // head dim (bf16 path)
 constexpr int kQTile = 64;      // query vectors per CTA
-constexpr int kRowBytes = kD * 2;
-constexpr int kTileBytes = kChunk * kRowBytes;  // 16 KB
+constexpr int kStages = 3;      // chunks in the ring (2 in flight while one is consumed)
+constexpr int kHalf = kChunk * 128;         // one [64 keys][64 d] bf16 half-tile: 8 KB
+constexpr int kStageBytes = 4 * kHalf;      // K lo, K hi, V lo, V hi: 32 KB
+constexpr int kPtCache = 512;               // page-table entries cached in shared memory
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-// byte offset of 16-byte column chunk c of row r in a swizzled [rows][128] bf16 tile
-__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * kRowBytes + ((c ^ (r & 7)) << 4)); }
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-    const int n = valid ? 16 : 0;  // 0 source bytes: zero-fill
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+// Byte offset of 16-byte column chunk c (0..15) of key row r in a K or V tile held as two [64][64]
+// bf16 halves written by TMA with the 128-byte swizzle (chunk c & 7 of row r sits at (c & 7) ^ (r & 7)).
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+    return (uint32_t)((c >> 3) * kHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -76,20 +79,75 @@ struct Unit {
     int b, g, qt, P, row_base, n_rows, nq, q0;
 };
 
+// Issue the TMA copies of chunk `ci` into stage `st` (one thread).  Prefix chunks copy whole pages
+// (64 / S pages, each as K and V halves); the last chunk copies the block's B cache rows.  Pages past
+// the prefix or with an out-of-range id are skipped (their keys stay masked).  Returns the valid-key
+// mask of the chunk.
+__device__ __forceinline__ uint64_t issue_chunk(const AttnArgs& a, const Unit& u, const CUtensorMap* pool_map,
+                                                const CUtensorMap* ibc_map, uint8_t* stage, uint64_t* bar, int ci,
+                                                int n_prefix_chunks, const int32_t* pt) {
+    const int S = a.page_size;
+    uint64_t mask = 0;
+    if (ci < n_prefix_chunks) {
+        uint32_t bytes = 0;
+        for (int p = 0; p < kChunk / S; ++p) {
+            const int t0 = ci * kChunk + p * S;
+            if (t0 >= u.P) break;
+            const int page = pt[t0 / S];
+            if (page < 0 || page >= a.n_pages) {
+                raise_err(a.err, FOCUS_DEVERR_PAGE_ID);
+                continue;
+            }
+            bytes += 4u * S * 128u;
+            const int n = min(S, u.P - t0);
+            mask |= (n == 64 ? ~0ull : ((1ull << n) - 1ull)) << (p * S);
+        }
+        mbar_expect_tx(bar, bytes);
+        for (int p = 0; p < kChunk / S; ++p) {
+            const int t0 = ci * kChunk + p * S;
+            if (t0 >= u.P) break;
+            const int page = pt[t0 / S];
+            if (page < 0 || page >= a.n_pages) continue;
+            const int krow = (int)(((((size_t)page * a.L + a.layer) * 2 + 0) * a.Hkv + u.g) * S);
+            const int vrow = krow + a.Hkv * S;
+            uint8_t* dst = stage + p * S * 128;
+            tma_load_2d(pool_map, bar, dst, 0, krow);
+            tma_load_2d(pool_map, bar, dst + kHalf, 64, krow);
+            tma_load_2d(pool_map, bar, dst + 2 * kHalf, 0, vrow);
+            tma_load_2d(pool_map, bar, dst + 3 * kHalf, 64, vrow);
+        }
+    } else {
+        const int krow = (int)(((((size_t)u.b * a.L + a.layer) * 2 + 0) * a.Hkv + u.g) * a.B);
+        const int vrow = krow + a.Hkv * a.B;
+        mbar_expect_tx(bar, 4u * a.B * 128u);
+        tma_load_2d(ibc_map, bar, stage, 0, krow);
+        tma_load_2d(ibc_map, bar, stage + kHalf, 64, krow);
+        tma_load_2d(ibc_map, bar, stage + 2 * kHalf, 0, vrow);
+        tma_load_2d(ibc_map, bar, stage + 3 * kHalf, 64, vrow);
+        mask = a.B == 64 ? ~0ull : ((1ull << a.B) - 1ull);
+    }
+    return mask;
+}
+
 template <bool FULL>
-__global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a, int q_tiles) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    // [0, 64K): K/V double buffer (stage s: K at 2s*16K, V at (2s+1)*16K); [64K, 80K): Q tile
-    uint8_t* kv = smem;
-    uint8_t* qs = smem + 4 * kTileBytes;
+__global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_constant__ CUtensorMap pool_map,
+                                                              const __grid_constant__ CUtensorMap ibc_map, AttnArgs a,
+                                                              int q_tiles) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* kv = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t full_bar[kStages];
+    __shared__ uint64_t valid_s[kStages];
     __shared__ float ml_s[4][16][2];      // per warp: row max / denominator (log2 domain)
     __shared__ float col_s[4][kChunk];    // per row tile: block-key column sums
+    __shared__ int32_t pt_s[kPtCache];     // this request's page-table row
+    __shared__ float fin_s[kQTile][2];     // split merge: final row max / denominator
+    __shared__ int last_s;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.Hq / a.Hkv;
     Unit u;
     u.b = blockIdx.x;
-    u.g = blockIdx.y;
+    u.g = blockIdx.y % a.Hkv;
     u.qt = blockIdx.z;
     u.P = checked_prefix(a.prefix_len, u.b, a.max_pages * a.page_size, a.err);
     if (FULL) {
@@ -107,84 +165,67 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a, int q_
     const int rt = warp % RT, ks = warp / RT;
     const int keys_per_warp = kChunk / KS;  // 64, 32 or 16
     const int key0 = ks * keys_per_warp;
-
-    const bf16* qg = reinterpret_cast<const bf16*>(a.q);
-    const bf16* pool = reinterpret_cast<const bf16*>(a.kv_pool);
-    const bf16* ibc = reinterpret_cast<const bf16*>(a.ibc);
-    const size_t ibc_k = ((((size_t)u.b * a.L + a.layer) * 2 + 0) * a.Hkv + u.g) * (size_t)a.B * kD;
-    const size_t ibc_v = ((((size_t)u.b * a.L + a.layer) * 2 + 1) * a.Hkv + u.g) * (size_t)a.B * kD;
     const int n_prefix_chunks = (u.P + kChunk - 1) / kChunk;
     const int n_chunks = n_prefix_chunks + 1;
+    // split-KV: this CTA walks chunks [c_begin, c_end) of the unit's n_chunks
+    const int pieces = a.pieces;  // grid.y = Hkv * pieces
+    const int cpp = (n_chunks + pieces - 1) / pieces;
+    const int piece = blockIdx.y / a.Hkv;
+    const int c_begin = piece * cpp, c_end = min(n_chunks, c_begin + cpp);
+    if (c_begin >= c_end) return;
+    const int n_active = (n_chunks + cpp - 1) / cpp;
+    const int unit = (u.b * a.Hkv + u.g) * q_tiles + u.qt;
 
-    // ---- Q tile -> shared (rows beyond nq zero-filled)
-    for (int i = threadIdx.x; i < kQTile * 16; i += 128) {
-        const int r = i >> 4, c = i & 15;
-        const int qi = u.q0 + r;
-        const bool ok = r < u.nq;
-        const int row = qi / G, hh = u.g * G + (qi - (qi / G) * G);
-        const bf16* src = qg + ((size_t)(u.row_base + (ok ? row : 0)) * a.Hq + (ok ? hh : 0)) * kD + c * 8;
-        cp_async16(smem_u32(qs) + swz(r, c), src, ok);
+    // page-table row -> shared (one latency for the whole CTA instead of one per issued chunk)
+    const bool pt_cached = a.max_pages <= kPtCache;
+    for (int i = threadIdx.x; pt_cached && i < a.max_pages; i += 128)
+        pt_s[i] = a.page_table[(size_t)u.b * a.max_pages + i];
+    const int32_t* pt = pt_cached ? pt_s : a.page_table + (size_t)u.b * a.max_pages;
+
+    // zero the ring once: skipped pages and short blocks then leave finite values behind masked keys
+    {
+        uint4* z = reinterpret_cast<uint4*>(kv);
+        for (int i = threadIdx.x; i < kStages * kStageBytes / 16; i += 128) z[i] = make_uint4(0, 0, 0, 0);
     }
-    // ---- chunk loader: K and V rows of chunk `ci` into stage `st`
-    auto load_chunk = [&](int ci, int st) {
-        const uint32_t kdst = smem_u32(kv) + (2 * st) * kTileBytes;
-        const uint32_t vdst = kdst + kTileBytes;
-        for (int i = threadIdx.x; i < kChunk * 16; i += 128) {
-            const int r = i >> 4, c = i & 15;
-            const bf16* ks_src = pool;
-            const bf16* vs_src = pool;
-            bool ok;
-            if (ci < n_prefix_chunks) {
-                const int t = ci * kChunk + r;
-                ok = t < u.P;
-                if (ok) {
-                    const int page = a.page_table[(size_t)u.b * a.max_pages + t / a.page_size];
-                    if (page < 0 || page >= a.n_pages) {
-                        raise_err(a.err, FOCUS_DEVERR_PAGE_ID);
-                        ok = false;
-                    } else {
-                        const size_t base = ((((size_t)page * a.L + a.layer) * 2) * a.Hkv + u.g) * (size_t)a.page_size * kD +
-                                            (size_t)(t % a.page_size) * kD + c * 8;
-                        ks_src = pool + base;
-                        vs_src = pool + base + (size_t)a.Hkv * a.page_size * kD;
-                    }
-                }
-            } else {
-                ok = r < a.B;
-                if (ok) {
-                    ks_src = ibc + ibc_k + (size_t)r * kD + c * 8;
-                    vs_src = ibc + ibc_v + (size_t)r * kD + c * 8;
-                }
-            }
-            cp_async16(kdst + swz(r, c), ks_src, ok);
-            cp_async16(vdst + swz(r, c), vs_src, ok);
-        }
-    };
-    auto key_valid = [&](int ci, int key) -> bool {
-        if (ci < n_prefix_chunks) {
-            const int t = ci * kChunk + key;
-            if (t >= u.P) return false;
-            const int page = a.page_table[(size_t)u.b * a.max_pages + t / a.page_size];
-            return page >= 0 && page < a.n_pages;
-        }
-        return key < a.B;
-    };
-
-    load_chunk(0, 0);
-    cp_commit();
-
-    // ---- Q fragments (A operand) for this warp's 16 rows, all 8 k-steps of d
-    cp_wait<0>();
+    if (threadIdx.x == 0) {
+        for (int s2 = 0; s2 < kStages; ++s2) mbar_init(&full_bar[s2], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
     __syncthreads();
+    int issued = 0;  // chunks whose copies thread 0 has issued
+    if (threadIdx.x == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // zeros before the TMA writes
+        for (int i = 0; i < kStages - 1 && c_begin + i < c_end; ++i) {
+            valid_s[i] = issue_chunk(a, u, &pool_map, &ibc_map, kv + i * kStageBytes, &full_bar[i], c_begin + i,
+                                     n_prefix_chunks, pt);
+            ++issued;
+        }
+    }
+
+    // ---- Q fragments (A operand) of this warp's 16 query vectors, straight from global memory
+    const int gq = lane >> 2, tq = lane & 3;
     uint32_t qf[8][4];
     {
-        const int r = rt * 16 + (lane & 15);
+        const bf16* qg = reinterpret_cast<const bf16*>(a.q);
+        const uint32_t* rowp[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int v = rt * 16 + gq + 8 * h;
+            const int qi = u.q0 + (v < u.nq ? v : 0);
+            const int row = qi / G, hh = u.g * G + (qi - row * G);
+            rowp[h] = v < u.nq ? reinterpret_cast<const uint32_t*>(qg + ((size_t)(u.row_base + row) * a.Hq + hh) * kD)
+                               : nullptr;
+        }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            const int c = kk * 2 + (lane >> 4);
-            ldsm_x4(smem_u32(qs) + swz(r, c), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+            const int c = kk * 8 + tq;  // 32-bit word: columns 16 kk + 2 tq, +1
+            qf[kk][0] = rowp[0] ? rowp[0][c] : 0u;
+            qf[kk][1] = rowp[1] ? rowp[1][c] : 0u;
+            qf[kk][2] = rowp[0] ? rowp[0][c + 4] : 0u;
+            qf[kk][3] = rowp[1] ? rowp[1][c + 4] : 0u;
         }
     }
+    __syncthreads();  // valid_s of the first chunks
     const float sl2 = rsqrtf((float)kD) * 1.4426950408889634f;  // 1/sqrt(d) * log2(e)
     float m_r[2] = {-CUDART_INF_F, -CUDART_INF_F}, l_r[2] = {0.f, 0.f};
     float o[16][4];
@@ -194,15 +235,24 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a, int q_
 #pragma unroll
     for (int n = 0; n < 8; ++n) sb[n][0] = sb[n][1] = sb[n][2] = sb[n][3] = -CUDART_INF_F;
 
-    const int gq = lane >> 2, tq = lane & 3;
-    for (int ci = 0; ci < n_chunks; ++ci) {
-        const int st = ci & 1;
-        if (ci + 1 < n_chunks) load_chunk(ci + 1, st ^ 1);
-        cp_commit();
-        cp_wait<1>();
-        __syncthreads();
-        const uint32_t kbase = smem_u32(kv) + (2 * st) * kTileBytes;
-        const uint32_t vbase = kbase + kTileBytes;
+    bool alive = true;
+    for (int ci = c_begin; ci < c_end; ++ci) {
+        const int i = ci - c_begin;       // position in this CTA's ring
+        const int st = i % kStages;
+        if (threadIdx.x == 0 && ci + kStages - 1 < c_end) {
+            const int sn = (i + kStages - 1) % kStages;  // stage of chunk ci - 1: free since the last sync
+            valid_s[sn] = issue_chunk(a, u, &pool_map, &ibc_map, kv + sn * kStageBytes, &full_bar[sn],
+                                      ci + kStages - 1, n_prefix_chunks, pt);
+            ++issued;
+        }
+        const bool landed = mbar_wait(&full_bar[st], (uint32_t)(i / kStages) & 1u, a.err);
+        if (__syncthreads_or(!landed)) {  // block-uniform: nobody is left waiting at a barrier
+            alive = false;
+            break;
+        }
+        const uint64_t vmask = valid_s[st];
+        const uint32_t kbase = smem_u32(kv + st * kStageBytes);
+        const uint32_t vbase = kbase + 2 * kHalf;
         // S = Q K^T over this warp's key slice: keys_per_warp / 8 n-tiles (up to 8)
         float s[8][4];
         const int n_nt = keys_per_warp / 8;
@@ -229,7 +279,7 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a, int q_
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int key = key0 + n * 8 + 2 * tq + (e & 1);
-                const float v = key_valid(ci, key) ? s[n][e] * sl2 : -CUDART_INF_F;
+                const float v = ((vmask >> key) & 1ull) ? s[n][e] * sl2 : -CUDART_INF_F;
                 s[n][e] = v;
                 mx[e >> 1] = fmaxf(mx[e >> 1], v);
             }
@@ -293,9 +343,16 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a, int q_
                 mma16816(o[2 * dp + 1], pa0, pa1, pa2, pa3, b2, b3);
             }
         }
-        __syncthreads();  // stage st is refilled by the next iteration's prefetch
+        __syncthreads();  // stage st is refilled two iterations later
     }
-    cp_wait<0>();
+    if (!alive) {
+        // a copy never landed: wait (bounded) for the chunks still in the ring so that no TMA write
+        // lands in a CTA that has exited; the outputs of this unit stay unwritten (error flagged)
+        if (threadIdx.x == 0)
+            for (int c = issued - kStages < 0 ? 0 : issued - kStages; c < issued; ++c)
+                mbar_wait(&full_bar[c % kStages], (uint32_t)(c / kStages) & 1u, a.err);
+        return;
+    }
 
     // ---- merge the key slices: final M, L per row of each row tile
     if (tq == 0) {
@@ -318,8 +375,8 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a, int q_
         L[h] = ll;
         f[h] = exp2f(m_r[h] - mu);  // this slice's weight
     }
-    // o slices -> shared (fp32), summed by the ks == 0 warp of each row tile
-    float* osum = reinterpret_cast<float*>(smem);  // reuses the K/V buffers: [warps][16][128]
+    // o slices -> shared (fp32), summed over the key slices by the ks == 0 warp of each row tile
+    float* osum = reinterpret_cast<float*>(kv);  // reuses the ring: [warps][16][128]
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
         const int d0 = n * 8 + 2 * tq;
@@ -331,16 +388,23 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a, int q_
         r1[1] = o[n][3] * f[1];
     }
     __syncthreads();
+    const bool split = n_active > 1;
     if (ks == 0) {
         bf16* og = reinterpret_cast<bf16*>(a.o);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int r = gq + 8 * h;
-            const int qi = u.q0 + rt * 16 + r;
-            if (rt * 16 + r >= u.nq) continue;
-            const int row = qi / G, hh = u.g * G + (qi - (qi / G) * G);
+            const int v = rt * 16 + r;  // query vector within the tile
+            if (v >= u.nq) continue;
+            const int qi = u.q0 + v;
+            const int row = qi / G, hh = u.g * G + (qi - row * G);
             bf16* dst = og + ((size_t)(u.row_base + row) * a.Hq + hh) * kD;
             const float inv = L[h] > 0.f ? 1.f / L[h] : 0.f;
+            const size_t pofs = ((size_t)unit * a.pieces + piece) * kQTile + v;
+            if (split && tq == 0) {
+                a.part_ml[2 * pofs] = M[h];
+                a.part_ml[2 * pofs + 1] = L[h];
+            }
             for (int n = 0; n < 16; ++n) {
                 const int d0 = n * 8 + 2 * tq;
                 float v0 = 0.f, v1 = 0.f;
@@ -349,9 +413,78 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a, int q_
                     v0 += src[0];
                     v1 += src[1];
                 }
-                *reinterpret_cast<__nv_bfloat162*>(dst + d0) = __floats2bfloat162_rn(v0 * inv, v1 * inv);
+                if (split) {
+                    *reinterpret_cast<float2*>(a.part_o + pofs * kD + d0) = make_float2(v0, v1);
+                } else {
+                    *reinterpret_cast<__nv_bfloat162*>(dst + d0) = __floats2bfloat162_rn(v0 * inv, v1 * inv);
+                }
             }
         }
+    }
+    if (split) {
+        // the piece holding the block chunk leaves its raw block scores for the importance
+        if (FULL && a.imp_part != nullptr && c_end == n_chunks) {
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                if (n >= keys_per_warp / 8) continue;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int v = rt * 16 + gq + 8 * (e >> 1);
+                    const int key = key0 + n * 8 + 2 * tq + (e & 1);
+                    if (v < u.nq) a.sb_buf[((size_t)unit * kQTile + v) * kChunk + key] = sb[n][e];
+                }
+            }
+        }
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) last_s = atomicAdd(&a.counters[unit], 1) == n_active - 1;
+        __syncthreads();
+        if (!last_s) return;
+        __threadfence();
+        // last piece of the unit: merge the pieces in piece order (deterministic)
+        bf16* og = reinterpret_cast<bf16*>(a.o);
+        for (int v = warp; v < u.nq; v += 4) {
+            float mm = -CUDART_INF_F;
+            for (int p2 = 0; p2 < n_active; ++p2)
+                mm = fmaxf(mm, __ldcg(a.part_ml + 2 * (((size_t)unit * a.pieces + p2) * kQTile + v)));
+            const float mu = mm == -CUDART_INF_F ? 0.f : mm;
+            float ll = 0.f;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int p2 = 0; p2 < n_active; ++p2) {
+                const size_t pofs = ((size_t)unit * a.pieces + p2) * kQTile + v;
+                const float w = exp2f(__ldcg(a.part_ml + 2 * pofs) - mu);
+                ll += __ldcg(a.part_ml + 2 * pofs + 1) * w;
+                const float4 x = __ldcg(reinterpret_cast<const float4*>(a.part_o + pofs * kD) + lane);
+                acc[0] += x.x * w;
+                acc[1] += x.y * w;
+                acc[2] += x.z * w;
+                acc[3] += x.w * w;
+            }
+            if (lane == 0) {
+                fin_s[v][0] = mu;
+                fin_s[v][1] = ll;
+            }
+            const float inv = ll > 0.f ? 1.f / ll : 0.f;
+            const int qi = u.q0 + v;
+            const int row = qi / G, hh = u.g * G + (qi - row * G);
+            bf16* dst = og + ((size_t)(u.row_base + row) * a.Hq + hh) * kD + lane * 4;
+            *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+            *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) a.counters[unit] = 0;  // ready for the next launch
+        if constexpr (FULL) {
+            if (a.imp_part == nullptr) return;
+            for (int j = threadIdx.x; j < a.B; j += 128) {
+                float col = 0.f;
+                for (int v = 0; v < u.nq; ++v) {
+                    const float sv = __ldcg(a.sb_buf + ((size_t)unit * kQTile + v) * kChunk + j);
+                    if (sv != -CUDART_INF_F && fin_s[v][1] > 0.f) col += exp2f(sv - fin_s[v][0]) / fin_s[v][1];
+                }
+                a.imp_part[(size_t)unit * a.B + j] = col;
+            }
+        }
+        return;
     }
     if constexpr (FULL) {
     if (a.imp_part == nullptr) return;
@@ -391,26 +524,66 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(AttnArgs a, int q_
     for (int j = threadIdx.x; j < a.B; j += 128) {
         float v = 0.f;
         for (int t = 0; t < RT; ++t) v += col_s[t][j];
-        a.imp_part[(((size_t)u.b * a.Hkv + u.g) * q_tiles + u.qt) * a.B + j] = v;
+        a.imp_part[(size_t)unit * a.B + j] = v;
     }
     }  // FULL
 }
 
 }  // namespace
 
+bool configure_attention_tc_kernels() {
+    return max_shared_carveout((const void*)attention_tc_kernel<true>) &&
+           max_shared_carveout((const void*)attention_tc_kernel<false>);
+}
+
 int attention_q_tiles(int B, int G) { return (B * G + kQTile - 1) / kQTile; }
+
+bool attention_tc_page_size_ok(int S) { return S == 16 || S == 32 || S == 64; }
+
+int attention_pieces(int units, int max_chunks) {
+    // aim at about four resident CTAs per SM-slot pair (148 SMs x 2 CTAs x 2) so that no single long
+    // request walk sets the kernel's duration; capped by the split scratch
+    constexpr int kTargetCtas = 4 * 148;
+    // with at least one unit per SM the walks are long-lived streams already: splitting them only adds
+    // start-up and merge cost per piece (measured), so only few-unit launches are split
+    if (units <= 0 || units >= 148 || units > kAttnSplitCap) return 1;
+    int p = (kTargetCtas + units - 1) / units;
+    if (p > max_chunks) p = max_chunks;
+    if (p > kAttnSplitCap / units) p = kAttnSplitCap / units;
+    return p < 1 ? 1 : p;
+}
 
 int launch_attention_tc(const AttnArgs& a, int q_tiles, cudaStream_t s) {
     if (a.N <= 0 || q_tiles <= 0) return 0;
-    const int smem = 4 * kTileBytes + kQTile * kRowBytes;  // 80 KB
-    dim3 grid(a.N, a.Hkv, q_tiles);
-    if (a.row_offsets == nullptr) {
-        cudaFuncSetAttribute(attention_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        attention_tc_kernel<true><<<grid, 128, smem, s>>>(a, q_tiles);
+    // 2-D views for TMA: every (page, layer, K|V, head) block of S rows and every (request, layer,
+    // K|V, head) cache block of B rows is a run of consecutive 256-byte rows
+    CUtensorMap pool_map, ibc_map;
+    const uint64_t ibc_rows = (uint64_t)a.N * a.L * 2 * a.Hkv * a.B;
+    if (!tc::make_map(&ibc_map, a.ibc, ibc_rows, kD, (uint32_t)a.B)) return -1;
+    if (a.n_pages > 0) {
+        const uint64_t pool_rows = (uint64_t)a.n_pages * a.L * 2 * a.Hkv * a.page_size;
+        if (!tc::make_map(&pool_map, a.kv_pool, pool_rows, kD, (uint32_t)a.page_size)) return -1;
     } else {
-        cudaFuncSetAttribute(attention_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        attention_tc_kernel<false><<<grid, 128, smem, s>>>(a, q_tiles);
+        pool_map = ibc_map;  // never used: with no pages every prefix key is invalid
     }
+    const int smem = kStages * kStageBytes + 1024;  // 97 KB: two CTAs per SM
+    // the shared-memory opt-in is set once per device (not per launch, so launches stay capturable)
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(attention_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(attention_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess)
+            return -1;
+        attr_set[dev] = true;
+    }
+    dim3 grid(a.N, a.Hkv * a.pieces, q_tiles);
+    if (a.row_offsets == nullptr)
+        attention_tc_kernel<true><<<grid, 128, smem, s>>>(pool_map, ibc_map, a, q_tiles);
+    else
+        attention_tc_kernel<false><<<grid, 128, smem, s>>>(pool_map, ibc_map, a, q_tiles);
     return 1;
 }
 

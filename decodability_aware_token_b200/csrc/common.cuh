@@ -43,6 +43,70 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
     return t;
 }
 
+template <typename T> __device__ __forceinline__ void store4(T* p, float a, float b, float c, float d);
+template <> __device__ __forceinline__ void store4<float>(float* p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+template <> __device__ __forceinline__ void store4<bf16>(bf16* p, float a, float b, float c, float d) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&lo);
+    u.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+template <typename T> __device__ __forceinline__ float4 load4(const T* p);
+template <> __device__ __forceinline__ float4 load4<float>(const float* p) { return *reinterpret_cast<const float4*>(p); }
+template <> __device__ __forceinline__ float4 load4<bf16>(const bf16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+// RMSNorm of one float32 row by one CTA of kNormThreads threads.  Thread t holds the row's float4
+// number i * kNormThreads + t in v[i] (i < kNormVec, D % 4 == 0, D <= 4 * kNormThreads * kNormVec);
+// the gamma loads are issued before the reduction so that the row costs two memory round trips.
+// h = x / sqrt(mean(x^2) + eps) * gamma.  Every kernel that normalises a residual row goes through
+// this routine, so all of them produce bit-identical results.  Contains __syncthreads().
+constexpr int kNormThreads = 256;
+constexpr int kNormVec = 4;  // D <= 4096
+template <typename T>
+__device__ __forceinline__ void rmsnorm_finish_cta(const float4 (&v)[kNormVec], int D, const T* gamma, float eps,
+                                                   T* hr, float* red) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float4 g[kNormVec];
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+        const int c = (i * kNormThreads + tid) * 4;
+        g[i] = c < D ? load4<T>(gamma + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+        const int c = (i * kNormThreads + tid) * 4;
+        if (c < D) {
+            ss = fmaf(v[i].x, v[i].x, ss);
+            ss = fmaf(v[i].y, v[i].y, ss);
+            ss = fmaf(v[i].z, v[i].z, ss);
+            ss = fmaf(v[i].w, v[i].w, ss);
+        }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kNormThreads / 32; ++w) tot += red[w];  // fixed order: deterministic
+    const float inv = rsqrtf(tot / D + eps);
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+        const int c = (i * kNormThreads + tid) * 4;
+        if (c < D)
+            store4<T>(hr + c, __fmul_rn(__fmul_rn(v[i].x, inv), g[i].x), __fmul_rn(__fmul_rn(v[i].y, inv), g[i].y),
+                      __fmul_rn(__fmul_rn(v[i].z, inv), g[i].z), __fmul_rn(__fmul_rn(v[i].w, inv), g[i].w));
+    }
+}
+
 // Where the rows of the current phase come from.
 //  full phase:      row r is block position (r / B, r % B)
 //  compacted phase: row r is (row_req[r], row_pos[r]); the live row count is *n_rows

@@ -1,4 +1,4 @@
-// LM-head combine + confidence-threshold decode.
+// LM-head combine (one CTA per kept row) + confidence-threshold decode (one CTA per request).
 //
 // The LM-head GEMM leaves, per kept row and vocabulary tile, the tile's max logit, the sum of
 // exp(z - tile max) and the first (lowest-id) argmax, so logits never reach HBM.  Merging the tiles
@@ -31,6 +31,57 @@ __device__ __forceinline__ void merge_stats(float& m, float& s, int& a, float m2
     }
 }
 
+// One CTA per kept row: merge the row's vocabulary-tile statistics into its confidence and top id.
+// Each thread loads its tiles (8 at a time, all in flight) before merging them; threads, then warps,
+// are merged in a fixed order.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineBatch = 8;
+__global__ void __launch_bounds__(kCombineThreads) lm_combine_kernel(const float* __restrict__ lm_max,
+                                                                     const float* __restrict__ lm_sum,
+                                                                     const int32_t* __restrict__ lm_arg, int n_tiles,
+                                                                     const int32_t* __restrict__ n_rows,
+                                                                     float* __restrict__ row_conf,
+                                                                     int32_t* __restrict__ row_top) {
+    __shared__ float wm[kCombineThreads / 32], ws[kCombineThreads / 32];
+    __shared__ int wa[kCombineThreads / 32];
+    const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (r >= *n_rows) return;
+    const size_t base = (size_t)r * n_tiles;
+    float m = -CUDART_INF_F, s = 0.f;
+    int arg = 0x7fffffff;
+    for (int t0 = 0; t0 < n_tiles; t0 += kCombineThreads * kCombineBatch) {
+        float bm[kCombineBatch], bs[kCombineBatch];
+        int ba[kCombineBatch];
+#pragma unroll
+        for (int i = 0; i < kCombineBatch; ++i) {
+            const int t = t0 + i * kCombineThreads + tid;
+            const bool ok = t < n_tiles;
+            bm[i] = ok ? lm_max[base + t] : -CUDART_INF_F;
+            bs[i] = ok ? lm_sum[base + t] : 0.f;
+            ba[i] = ok ? lm_arg[base + t] : 0x7fffffff;
+        }
+#pragma unroll
+        for (int i = 0; i < kCombineBatch; ++i) merge_stats(m, s, arg, bm[i], bs[i], ba[i]);
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        const int a2 = __shfl_xor_sync(0xffffffffu, arg, o);
+        merge_stats(m, s, arg, m2, s2, a2);
+    }
+    if (lane == 0) {
+        wm[warp] = m;
+        ws[warp] = s;
+        wa[warp] = arg;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        for (int w = 1; w < kCombineThreads / 32; ++w) merge_stats(m, s, arg, wm[w], ws[w], wa[w]);
+        row_conf[r] = 1.f / s;
+        row_top[r] = arg;
+    }
+}
+
 __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(DecodeArgs a) {
     __shared__ float conf_s[64];
     __shared__ int top_s[64];
@@ -38,23 +89,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(DecodeArgs a)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int k = a.keep_count[b], off = a.row_offsets[b], B = a.B;
     for (int j = threadIdx.x; j < B; j += blockDim.x) a.decoded_ids[(size_t)b * B + j] = -1;
-    for (int t = warp; t < k; t += kDecodeWarps) {
-        const size_t r = (size_t)(off + t);
-        float m = -CUDART_INF_F, s = 0.f;
-        int arg = 0x7fffffff;
-        for (int tile = lane; tile < a.n_tiles; tile += 32)
-            merge_stats(m, s, arg, a.lm_max[r * a.n_tiles + tile], a.lm_sum[r * a.n_tiles + tile],
-                        a.lm_arg[r * a.n_tiles + tile]);
-        for (int o = 16; o > 0; o >>= 1) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-            const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-            const int a2 = __shfl_xor_sync(0xffffffffu, arg, o);
-            merge_stats(m, s, arg, m2, s2, a2);
-        }
-        if (lane == 0) {
-            conf_s[t] = 1.f / s;
-            top_s[t] = arg;
-        }
+    for (int t = threadIdx.x; t < k; t += blockDim.x) {
+        conf_s[t] = a.row_conf[off + t];
+        top_s[t] = a.row_top[off + t];
     }
     __syncthreads();
     for (int t = threadIdx.x; t < a.max_keep; t += blockDim.x) {
@@ -104,6 +141,18 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(DecodeArgs a)
 }
 
 }  // namespace
+
+bool configure_select_decode_kernels() {
+    return configure_select_kernel() && max_shared_carveout((const void*)decode_kernel) &&
+           max_shared_carveout((const void*)lm_combine_kernel);
+}
+
+int launch_lm_combine(const DecodeArgs& a, int rows_bound, const int32_t* n_rows, cudaStream_t s) {
+    if (rows_bound <= 0) return 0;
+    lm_combine_kernel<<<rows_bound, kCombineThreads, 0, s>>>(a.lm_max, a.lm_sum, a.lm_arg, a.n_tiles, n_rows,
+                                                            a.row_conf, a.row_top);
+    return 1;
+}
 
 int launch_decode(const DecodeArgs& a, cudaStream_t s) {
     if (a.N <= 0) return 0;

@@ -36,6 +36,11 @@ struct focus_ctx {
     int32_t *row_req, *row_pos, *row_src, *n_rows, *lm_arg;
     double* inv_freq;
     int* err;
+    float *att_part_o, *att_part_ml, *att_sb;
+    int* att_counters;
+    int* gemm_counters;
+    float* row_conf;
+    int32_t* row_top;
     size_t part_rows;     // rows of the partial-sum buffer
     size_t split_stride;  // elements between split-K slices
     int lm_tiles_cap;
@@ -50,9 +55,10 @@ struct focus_ctx {
 namespace {
 
 constexpr int kMaxSplits = 8;
+constexpr int kGemmCounters = 1024;  // output tiles of one split-K GEMM launch (at most 2 x 48 here)
 
 struct Layout {
-    size_t off[20];
+    size_t off[32];
     size_t total;
 };
 
@@ -71,7 +77,7 @@ bool cfg_ok(const focus_model_cfg* c) {
 int shape_supported(const focus_model_cfg* c) {
     if (c->head_dim != 64 && c->head_dim != 128) return FOCUS_ERR_UNSUPPORTED;
     if (c->dtype == FOCUS_DTYPE_BF16 && c->head_dim != 128) return FOCUS_ERR_UNSUPPORTED;
-    if (c->hidden % 64 || c->ffn % 64) return FOCUS_ERR_UNSUPPORTED;
+    if (c->hidden % 128 || c->hidden > 4096 || c->ffn % 64) return FOCUS_ERR_UNSUPPORTED;
     return FOCUS_OK;
 }
 
@@ -95,6 +101,7 @@ Layout plan(const focus_model_cfg* c, const focus_limits* l) {
     const size_t qkv = (size_t)(c->n_q_heads + 2 * c->n_kv_heads) * c->head_dim;
     const size_t part_rows = rows_full > kMaxSplits * rows_c ? rows_full : kMaxSplits * rows_c;
     const size_t widest = qkv > D ? qkv : D;
+    const size_t split = c->dtype == FOCUS_DTYPE_BF16 ? 1 : 0;
     const size_t sizes[] = {
         rows_full * D * 4,                                  // 0 x_full
         rows_c * D * 4,                                     // 1 x_c
@@ -111,10 +118,16 @@ Layout plan(const focus_model_cfg* c, const focus_limits* l) {
         rows_c * lm_tiles(c) * 4,                           // 14 lm_arg
         (size_t)c->head_dim / 2 * 8,                        // 15 inv_freq
         64,                                                 // 16 err
+        split * (size_t)kAttnSplitCap * 64 * 128 * 4,       // 17 attention split partial outputs
+        split * (size_t)kAttnSplitCap * 64 * 2 * 4,         // 18 partial row max / denominator
+        split * (size_t)kAttnSplitCap * 64 * 64 * 4,        // 19 raw block scores
+        split * (size_t)kAttnSplitCap * 4,                  // 20 arrival counters
+        (size_t)kGemmCounters * 4,                          // 21 split-K GEMM tile counters
+        rows_c * 4, rows_c * 4,                             // 22-23 per-row confidence / top id
     };
     Layout lay{};
     size_t at = 0;
-    for (int i = 0; i < 17; ++i) {
+    for (int i = 0; i < 24; ++i) {
         lay.off[i] = at;
         at = align_up(at + sizes[i], 1024);
     }
@@ -161,21 +174,36 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
 
     // every launch goes through here: launch accounting and optional per-class event timing
     int launches = 0;
+    bool launch_failed = false;
+    // inside a stream capture the profiling pairs are recorded as external event nodes of the graph,
+    // so they time every replay; outside a capture they are plain records
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (c->prof_active) FOCUS_CUDA_TRY(cudaStreamIsCapturing(s, &cap));
+    const unsigned rec_flags = cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
     auto run = [&](int kclass, auto&& launch) {
         const bool timed = c->prof_active && c->prof_class == kclass && c->prof_n < c->prof_cap;
-        if (timed) cudaEventRecord(c->prof_ev[2 * c->prof_n], s);
-        launches += launch();
+        if (timed && cudaEventRecordWithFlags(c->prof_ev[2 * c->prof_n], s, rec_flags) != cudaSuccess)
+            launch_failed = true;
+        const int n = launch();
+        if (n < 0) launch_failed = true;
+        else launches += n;
         if (timed) {
-            cudaEventRecord(c->prof_ev[2 * c->prof_n + 1], s);
+            if (cudaEventRecordWithFlags(c->prof_ev[2 * c->prof_n + 1], s, rec_flags) != cudaSuccess)
+                launch_failed = true;
             ++c->prof_n;
         }
     };
     auto gemm = [&](int kclass, Epi epi, const void* A, const void* Bw, const void* B2, int Mb, const int32_t* Md,
-                    int Nn, int K, int splits, int wid, void* act_out) {
+                    int Nn, int K, int splits, int wid, void* act_out, float* resid = nullptr, int layer = 0,
+                    bool compact = false) {
         GemmArgs g{};
         g.A = A; g.B = Bw; g.B2 = B2; g.M_bound = Mb; g.M_dev = Md; g.N = Nn; g.K = K; g.splits = splits;
         g.part = c->part; g.split_stride = stride; g.act = act_out;
         g.lm_max = c->lm_max; g.lm_sum = c->lm_sum; g.lm_arg = c->lm_arg;
+        g.counters = c->gemm_counters; g.resid = resid; g.q_out = c->q; g.ibc = in->ibc;
+        g.row_req = compact ? c->row_req : nullptr; g.row_pos = compact ? c->row_pos : nullptr;
+        g.prefix_len = in->prefix_len; g.inv_freq = c->inv_freq; g.max_prefix = max_prefix; g.block = B;
+        g.n_layers = dm.L; g.layer = layer; g.Hq = dm.Hq; g.Hkv = dm.Hkv; g.err = c->err;
         run(kclass, [&] {
             if (tc) return tc_gemm(c->tc, epi, wid, g, s);
             g.n_tiles = (Nn + kSimtTileN - 1) / kSimtTileN;
@@ -188,6 +216,11 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
     at.q = c->q; at.o = c->o; at.kv_pool = in->kv_pool; at.ibc = in->ibc; at.prefix_len = in->prefix_len;
     at.page_table = in->page_table; at.N = N; at.B = B; at.L = dm.L; at.Hq = dm.Hq; at.Hkv = dm.Hkv; at.d = dm.d;
     at.max_pages = c->lim.max_pages_per_req; at.page_size = in->page_size; at.n_pages = in->n_pages; at.err = c->err;
+    at.part_o = c->att_part_o; at.part_ml = c->att_part_ml; at.sb_buf = c->att_sb; at.counters = c->att_counters;
+    const int max_chunks = (c->lim.max_pages_per_req * in->page_size + 63) / 64 + 1;
+    const int pieces_full = bf ? attention_pieces(N * dm.Hkv * qt_full, max_chunks) : 1;
+    const int pieces_kept = bf ? attention_pieces(N * dm.Hkv * qt_kept, max_chunks) : 1;
+    if (bf) FOCUS_CUDA_TRY(cudaMemsetAsync(c->att_counters, 0, (size_t)kAttnSplitCap * 4, s));
 
     const RowMap full{nullptr, nullptr, nullptr, rows_full, B};
     const RowMap comp{c->row_req, c->row_pos, c->n_rows, R_bound, B};
@@ -196,32 +229,42 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
         return launch_embed_norm<T>(in->block_tokens, rows_full, dm.V, W(c->embed), W(c->attn_norm[0]), dm.eps, dm.D,
                                     c->x_full, h, c->err, s);
     });
+    // tensor-core path: the GEMM epilogues apply RoPE + the cache write (QKV) and the residual adds
+    // (O, down) themselves, reducing split-K partials in the GEMM; the row kernels only normalise
+    if (tc) FOCUS_CUDA_TRY(cudaMemsetAsync(c->gemm_counters, 0, (size_t)kGemmCounters * 4, s));
     // ---- layers 0 and 1: full block, importance at both
     for (int l = 0; l < 2; ++l) {
-        gemm(FOCUS_K_GEMM_FULL_QKV, EPI_PARTIAL, c->h, c->wqkv[l], nullptr, rows_full, nullptr, dm.qkv, dm.D, 1, W_QKV,
-             nullptr);
-        run(FOCUS_K_QKV_FINALIZE, [&] {
-            return launch_qkv_finalize<T>(c->part, 1, stride, full, in->prefix_len, max_prefix, c->inv_freq, dm, l, q,
-                                          ibc, c->err, s);
-        });
+        if (tc) {
+            gemm(FOCUS_K_GEMM_FULL_QKV, EPI_QKV, c->h, c->wqkv[l], nullptr, rows_full, nullptr, dm.qkv, dm.D, 1,
+                 W_QKV, nullptr, nullptr, l, false);
+        } else {
+            gemm(FOCUS_K_GEMM_FULL_QKV, EPI_PARTIAL, c->h, c->wqkv[l], nullptr, rows_full, nullptr, dm.qkv, dm.D, 1,
+                 W_QKV, nullptr);
+            run(FOCUS_K_QKV_FINALIZE, [&] {
+                return launch_qkv_finalize<T>(c->part, 1, stride, full, in->prefix_len, max_prefix, c->inv_freq, dm,
+                                              l, q, ibc, c->err, s);
+            });
+        }
         at.layer = l;
         at.row_offsets = nullptr;
         at.imp_part = c->imp_part + (size_t)l * N * dm.Hkv * qt_full * B;
+        at.pieces = pieces_full;
         run(FOCUS_K_ATTN_SCORE, [&] { return attention(at, qt_full); });
-        gemm(FOCUS_K_GEMM_FULL_O, EPI_PARTIAL, c->o, c->wo[l], nullptr, rows_full, nullptr, dm.D, dm.Hq * dm.d, 1, W_O,
-             nullptr);
+        const int nsp_full = tc ? 0 : 1;  // partial slices the norm kernels still add (CUDA-core path)
+        gemm(FOCUS_K_GEMM_FULL_O, tc ? EPI_RESID : EPI_PARTIAL, c->o, c->wo[l], nullptr, rows_full, nullptr, dm.D,
+             dm.Hq * dm.d, 1, W_O, nullptr, c->x_full, l, false);
         run(FOCUS_K_ROW_NORM, [&] {
-            return launch_residual_norm<T>(c->x_full, nullptr, nullptr, rows_full, c->part, 1, stride, c->x_full,
+            return launch_residual_norm<T>(c->x_full, nullptr, nullptr, rows_full, c->part, nsp_full, stride, c->x_full,
                                            W(c->mlp_norm[l]), dm.eps, dm.D, h, s);
         });
         gemm(FOCUS_K_GEMM_FULL_GATEUP, EPI_SWIGLU, c->h, c->wgate[l], c->wup[l], rows_full, nullptr, dm.F, dm.D, 1,
              W_GATEUP, c->act);
-        gemm(FOCUS_K_GEMM_FULL_DOWN, EPI_PARTIAL, c->act, c->wdown[l], nullptr, rows_full, nullptr, dm.D, dm.F, 1,
-             W_DOWN, nullptr);
+        gemm(FOCUS_K_GEMM_FULL_DOWN, tc ? EPI_RESID : EPI_PARTIAL, c->act, c->wdown[l], nullptr, rows_full, nullptr,
+             dm.D, dm.F, 1, W_DOWN, nullptr, c->x_full, l, false);
         if (l == 0)
             run(FOCUS_K_ROW_NORM, [&] {
-                return launch_residual_norm<T>(c->x_full, nullptr, nullptr, rows_full, c->part, 1, stride, c->x_full,
-                                               W(c->attn_norm[1]), dm.eps, dm.D, h, s);
+                return launch_residual_norm<T>(c->x_full, nullptr, nullptr, rows_full, c->part, nsp_full, stride,
+                                               c->x_full, W(c->attn_norm[1]), dm.eps, dm.D, h, s);
             });
     }
     // ---- delta, budget, top-k, row map
@@ -237,7 +280,7 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
     // ---- gather the kept rows (folding in layer 1's MLP partial sums) and normalise for layer 2
     const void* g_next = dm.L > 2 ? c->attn_norm[2] : c->final_norm;
     run(FOCUS_K_ROW_NORM, [&] {
-        return launch_residual_norm<T>(c->x_full, c->row_src, c->n_rows, R_bound, c->part, 1, stride, c->x_c,
+        return launch_residual_norm<T>(c->x_full, c->row_src, c->n_rows, R_bound, c->part, tc ? 0 : 1, stride, c->x_c,
                                        W(g_next), dm.eps, dm.D, h, s);
     });
     // ---- layers 2..L-1 on the kept rows
@@ -245,29 +288,35 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
     const int sp_o = tc ? tc_splits(c->tc, W_O, R_bound) : 1;
     const int sp_dn = tc ? tc_splits(c->tc, W_DOWN, R_bound) : 1;
     for (int l = 2; l < dm.L; ++l) {
-        gemm(FOCUS_K_GEMM_QKV, EPI_PARTIAL, c->h, c->wqkv[l], nullptr, R_bound, c->n_rows, dm.qkv, dm.D, sp_qkv, W_QKV,
-             nullptr);
-        run(FOCUS_K_QKV_FINALIZE, [&] {
-            return launch_qkv_finalize<T>(c->part, sp_qkv, stride, comp, in->prefix_len, max_prefix, c->inv_freq, dm,
-                                          l, q, ibc, c->err, s);
-        });
+        if (tc) {
+            gemm(FOCUS_K_GEMM_QKV, EPI_QKV, c->h, c->wqkv[l], nullptr, R_bound, c->n_rows, dm.qkv, dm.D, sp_qkv, W_QKV,
+                 nullptr, nullptr, l, true);
+        } else {
+            gemm(FOCUS_K_GEMM_QKV, EPI_PARTIAL, c->h, c->wqkv[l], nullptr, R_bound, c->n_rows, dm.qkv, dm.D, sp_qkv,
+                 W_QKV, nullptr);
+            run(FOCUS_K_QKV_FINALIZE, [&] {
+                return launch_qkv_finalize<T>(c->part, sp_qkv, stride, comp, in->prefix_len, max_prefix, c->inv_freq,
+                                              dm, l, q, ibc, c->err, s);
+            });
+        }
         at.layer = l;
         at.row_offsets = out->row_offsets;
         at.imp_part = nullptr;
+        at.pieces = pieces_kept;
         run(FOCUS_K_ATTN_RAGGED, [&] { return attention(at, qt_kept); });
-        gemm(FOCUS_K_GEMM_O, EPI_PARTIAL, c->o, c->wo[l], nullptr, R_bound, c->n_rows, dm.D, dm.Hq * dm.d, sp_o, W_O,
-             nullptr);
+        gemm(FOCUS_K_GEMM_O, tc ? EPI_RESID : EPI_PARTIAL, c->o, c->wo[l], nullptr, R_bound, c->n_rows, dm.D,
+             dm.Hq * dm.d, sp_o, W_O, nullptr, c->x_c, l, true);
         run(FOCUS_K_ROW_NORM, [&] {
-            return launch_residual_norm<T>(c->x_c, nullptr, c->n_rows, R_bound, c->part, sp_o, stride, c->x_c,
+            return launch_residual_norm<T>(c->x_c, nullptr, c->n_rows, R_bound, c->part, tc ? 0 : sp_o, stride, c->x_c,
                                            W(c->mlp_norm[l]), dm.eps, dm.D, h, s);
         });
         gemm(FOCUS_K_GEMM_GATEUP, EPI_SWIGLU, c->h, c->wgate[l], c->wup[l], R_bound, c->n_rows, dm.F, dm.D, 1,
              W_GATEUP, c->act);
-        gemm(FOCUS_K_GEMM_DOWN, EPI_PARTIAL, c->act, c->wdown[l], nullptr, R_bound, c->n_rows, dm.D, dm.F, sp_dn,
-             W_DOWN, nullptr);
+        gemm(FOCUS_K_GEMM_DOWN, tc ? EPI_RESID : EPI_PARTIAL, c->act, c->wdown[l], nullptr, R_bound, c->n_rows, dm.D,
+             dm.F, sp_dn, W_DOWN, nullptr, c->x_c, l, true);
         const void* gn = l + 1 < dm.L ? c->attn_norm[l + 1] : c->final_norm;
         run(FOCUS_K_ROW_NORM, [&] {
-            return launch_residual_norm<T>(c->x_c, nullptr, c->n_rows, R_bound, c->part, sp_dn, stride, c->x_c,
+            return launch_residual_norm<T>(c->x_c, nullptr, c->n_rows, R_bound, c->part, tc ? 0 : sp_dn, stride, c->x_c,
                                            W(gn), dm.eps, dm.D, h, s);
         });
     }
@@ -280,8 +329,11 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
     da.max_keep = c->lim.max_keep; da.tokens = in->block_tokens; da.mask = in->mask; da.N = N; da.B = B;
     da.threshold = p->conf_threshold; da.decoded_ids = out->decoded_ids; da.conf_out = out->conf;
     da.top_out = out->top_id;
+    da.row_conf = c->row_conf; da.row_top = c->row_top;
+    run(FOCUS_K_DECODE, [&] { return launch_lm_combine(da, R_bound, c->n_rows, s); });
     run(FOCUS_K_DECODE, [&] { return launch_decode(da, s); });
     c->last_launches = launches;
+    if (launch_failed) return FOCUS_ERR_CUDA;
     if (out->hidden && R_bound > 0)
         FOCUS_CUDA_TRY(cudaMemcpyAsync(out->hidden, c->x_c, (size_t)R_bound * dm.D * sizeof(float),
                                        cudaMemcpyDeviceToDevice, s));
@@ -377,6 +429,13 @@ int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_l
     c->lm_arg = reinterpret_cast<int32_t*>(base + lay.off[14]);
     c->inv_freq = reinterpret_cast<double*>(base + lay.off[15]);
     c->err = reinterpret_cast<int*>(base + lay.off[16]);
+    c->att_part_o = reinterpret_cast<float*>(base + lay.off[17]);
+    c->att_part_ml = reinterpret_cast<float*>(base + lay.off[18]);
+    c->att_sb = reinterpret_cast<float*>(base + lay.off[19]);
+    c->att_counters = reinterpret_cast<int*>(base + lay.off[20]);
+    c->gemm_counters = reinterpret_cast<int*>(base + lay.off[21]);
+    c->row_conf = reinterpret_cast<float*>(base + lay.off[22]);
+    c->row_top = reinterpret_cast<int32_t*>(base + lay.off[23]);
     const size_t rows_full = (size_t)lim->max_requests * lim->max_block;
     const size_t rows_c = (size_t)lim->max_requests * lim->max_keep;
     c->part_rows = rows_full > kMaxSplits * rows_c ? rows_full : kMaxSplits * rows_c;
@@ -388,7 +447,13 @@ int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_l
         inv[i] = pow((double)cfg->rope_theta, -2.0 * i / (double)cfg->head_dim);
     int rc = FOCUS_OK;
     if (cudaMemcpy(c->inv_freq, inv.data(), inv.size() * sizeof(double), cudaMemcpyHostToDevice) != cudaSuccess ||
-        cudaMemset(c->err, 0, sizeof(int)) != cudaSuccess || cudaMemset(c->n_rows, 0, sizeof(int)) != cudaSuccess)
+        cudaMemset(c->err, 0, sizeof(int)) != cudaSuccess || cudaMemset(c->n_rows, 0, sizeof(int)) != cudaSuccess ||
+        cudaMemset(c->gemm_counters, 0, (size_t)kGemmCounters * 4) != cudaSuccess ||
+        (cfg->dtype == FOCUS_DTYPE_BF16 &&
+         cudaMemset(c->att_counters, 0, (size_t)kAttnSplitCap * 4) != cudaSuccess))
+        rc = FOCUS_ERR_CUDA;
+    if (rc == FOCUS_OK && !(configure_rows_kernels() && configure_attention_kernels() &&
+                            configure_select_decode_kernels() && configure_simt_gemm_kernels()))
         rc = FOCUS_ERR_CUDA;
     c->tc = nullptr;
     if (rc == FOCUS_OK && cfg->dtype == FOCUS_DTYPE_BF16) {
@@ -435,6 +500,7 @@ int focus_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus
         if (p->k_max > c->lim.max_keep) return FOCUS_ERR_LIMITS;
         k_cap = p->k_max;
     }
+    if (c->cfg.dtype == FOCUS_DTYPE_BF16 && !attention_tc_page_size_ok(in->page_size)) return FOCUS_ERR_UNSUPPORTED;
     if (N == 0) return FOCUS_OK;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev != c->device) return FOCUS_ERR_INVALID_ARG;

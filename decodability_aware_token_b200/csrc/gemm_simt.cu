@@ -122,6 +122,15 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs g) {
 
 }  // namespace
 
+bool configure_simt_gemm_kernels() {
+    return max_shared_carveout((const void*)gemm_simt_kernel<float, EPI_PARTIAL>) &&
+           max_shared_carveout((const void*)gemm_simt_kernel<float, EPI_SWIGLU>) &&
+           max_shared_carveout((const void*)gemm_simt_kernel<float, EPI_LMHEAD>) &&
+           max_shared_carveout((const void*)gemm_simt_kernel<bf16, EPI_PARTIAL>) &&
+           max_shared_carveout((const void*)gemm_simt_kernel<bf16, EPI_SWIGLU>) &&
+           max_shared_carveout((const void*)gemm_simt_kernel<bf16, EPI_LMHEAD>);
+}
+
 template <typename T>
 int launch_gemm_simt(Epi epi, const GemmArgs& g, cudaStream_t s) {
     if (g.M_bound <= 0) return 0;

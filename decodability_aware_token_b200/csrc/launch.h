@@ -8,6 +8,20 @@
 
 namespace focus {
 
+// Every kernel of the step asks for the largest shared-memory carveout, so consecutive kernels never
+// need the SMs to drain and reconfigure the L1 / shared split between them.  The configure_* functions
+// set it (for the current device) at init and return false if an attribute could not be set.
+inline bool max_shared_carveout(const void* fn) {
+    return cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+}
+bool configure_rows_kernels();
+bool configure_attention_kernels();
+bool configure_attention_tc_kernels();
+bool configure_select_decode_kernels();
+bool configure_select_kernel();
+bool configure_simt_gemm_kernels();
+
 struct Dims {
     int L, D, Hq, Hkv, d, F, V, qkv;  // qkv = (Hq + 2 Hkv) d
     float eps;
@@ -45,12 +59,25 @@ struct AttnArgs {
     int N, B, layer, L, Hq, Hkv, d;
     int max_pages, page_size, n_pages;
     int* err;
+    // split-KV (tensor-core kernel): each (request, KV head, query tile) unit is walked by `pieces` CTAs;
+    // pieces > 1 needs the scratch below for units * pieces <= split_cap (and units <= split_cap)
+    int pieces;
+    float* part_o;              // [unit * pieces + piece][64][128] unnormalised partial outputs
+    float* part_ml;             // [unit * pieces + piece][64][2] partial row max / denominator (log2 domain)
+    float* sb_buf;              // [unit][64][64] raw block-key scores (layers 0-1)
+    int* counters;              // [unit] arrival counters, zero between launches
 };
+
+constexpr int kAttnSplitCap = 1280;  // unit-pieces the split-KV scratch holds
+// pieces for a launch of `units` work units whose longest key walk is `max_chunks` 64-key chunks
+int attention_pieces(int units, int max_chunks);
 template <typename T> int launch_attention(const AttnArgs& a, cudaStream_t s);
 // bf16, head_dim 128: tensor-core kernel (attention_tc.cu); the full phase writes its importance column
 // sums per (KV head, 64-vector query tile): imp_part [N, Hkv, q_tiles, B]
+// Returns the number of launches, or -1 if a tensor map could not be built.
 int launch_attention_tc(const AttnArgs& a, int q_tiles, cudaStream_t s);
 int attention_q_tiles(int B, int G);
+bool attention_tc_page_size_ok(int page_size);  // KV page sizes the TMA page loader handles: 16, 32, 64
 
 // ---- selection + compaction metadata (select.cu) ------------------------------
 struct SelectArgs {
@@ -74,7 +101,7 @@ struct SelectArgs {
 int launch_select(const SelectArgs& a, cudaStream_t s);
 
 // ---- GEMM C = A B^T with fused epilogues (gemm_simt.cu, gemm_tc.cu) -------------
-enum Epi { EPI_PARTIAL = 0, EPI_SWIGLU = 1, EPI_LMHEAD = 2 };
+enum Epi { EPI_PARTIAL = 0, EPI_SWIGLU = 1, EPI_LMHEAD = 2, EPI_RESID = 3, EPI_QKV = 4 };
 
 struct GemmArgs {
     const void* A;              // [M, K] row-major
@@ -92,6 +119,18 @@ struct GemmArgs {
     int32_t* lm_arg;
     int n_tiles;
     int tile_n;                 // EPI_LMHEAD: columns per stats tile
+    // tcgen05 fused epilogues (split K: every split writes its partial tile to `part`, and the last split
+    // CTA of each output tile -- counted in `counters`, zero between launches -- sums them in split order)
+    int* counters;
+    float* resid;               // EPI_RESID: [rows, N] float32 residual stream, resid += A B^T
+    void* q_out;                // EPI_QKV: [rows, Hq d] rotated queries (bf16)
+    void* ibc;                  // EPI_QKV: intra-block KV cache [N, L, 2, Hkv, B, d]: rotated K and V at (b, j)
+    const int32_t* row_req;     // EPI_QKV: compacted rows -> request / block position (null: row = b * B + j)
+    const int32_t* row_pos;
+    const int32_t* prefix_len;
+    const double* inv_freq;     // [d / 2] RoPE frequencies
+    int max_prefix, block, n_layers, layer, Hq, Hkv;
+    int* err;
 };
 template <typename T> int launch_gemm_simt(Epi epi, const GemmArgs& g, cudaStream_t s);
 constexpr int kSimtTileN = 64;
@@ -113,7 +152,10 @@ struct DecodeArgs {
     int32_t* decoded_ids;
     float* conf_out;
     int32_t* top_out;
+    float* row_conf;            // [R_max] per kept row: confidence (written by the combine kernel)
+    int32_t* row_top;           // [R_max] per kept row: top id
 };
+int launch_lm_combine(const DecodeArgs& a, int rows_bound, const int32_t* n_rows, cudaStream_t s);
 int launch_decode(const DecodeArgs& a, cudaStream_t s);
 
 }  // namespace focus

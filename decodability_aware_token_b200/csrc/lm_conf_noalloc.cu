@@ -37,23 +37,20 @@ static __device__ __align__(256) unsigned char g_lm_conf_scratch[kNaBytes];
 
 using NaShape = TcShape<kNaBN, 2, 4>;
 
-// RMSNorm of float32 rows into bf16; the same arithmetic (thread layout, reduction order) as the
-// step's residual / norm kernel, so both paths produce bit-identical normalised rows.
-__global__ void __launch_bounds__(256) na_norm_kernel(const float* __restrict__ x, int D,
-                                                      const bf16* __restrict__ gamma, float eps,
-                                                      bf16* __restrict__ h) {
+// RMSNorm of float32 rows into bf16, one CTA per row, with the very routine the step's own norm
+// kernels use, so both paths produce bit-identical normalised rows.
+__global__ void __launch_bounds__(kNormThreads) na_norm_kernel(const float* __restrict__ x, int D,
+                                                               const bf16* __restrict__ gamma, float eps,
+                                                               bf16* __restrict__ h) {
     __shared__ float red[32];
-    const int r = blockIdx.x;
-    const float* xr = x + (size_t)r * D;
-    float ss = 0.f;
-    for (int i = threadIdx.x; i < D; i += blockDim.x) {
-        const float v = xr[i];
-        ss += v * v;
+    const int r = blockIdx.x, tid = threadIdx.x;
+    float4 v[kNormVec];
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+        const int c = (i * kNormThreads + tid) * 4;
+        v[i] = c < D ? *reinterpret_cast<const float4*>(x + (size_t)r * D + c) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const float tot = block_sum(ss, red);
-    const float inv = rsqrtf(tot / D + eps);
-    bf16* hr = h + (size_t)r * D;
-    for (int i = threadIdx.x; i < D; i += blockDim.x) hr[i] = __float2bfloat16_rn(xr[i] * inv * __bfloat162float(gamma[i]));
+    rmsnorm_finish_cta<bf16>(v, D, gamma, eps, h + (size_t)r * D, red);
 }
 
 __device__ __forceinline__ void na_merge(float& m, float& s, int& a, float m2, float s2, int a2) {
@@ -104,7 +101,9 @@ int na_setup(int dev, void** base) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_lm_conf_scratch) != cudaSuccess || !p) return FOCUS_ERR_CUDA;
         if (cudaFuncSetAttribute(tc_gemm_kernel<kNaBN, 2, 4, EPI_LMHEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 NaShape::SMEM) != cudaSuccess)
+                                 NaShape::SMEM) != cudaSuccess ||
+            !max_shared_carveout((const void*)tc_gemm_kernel<kNaBN, 2, 4, EPI_LMHEAD>) ||
+            !max_shared_carveout((const void*)na_norm_kernel) || !max_shared_carveout((const void*)na_combine_kernel))
             return FOCUS_ERR_CUDA;
         g_na_base[dev] = p;
     }
@@ -125,7 +124,7 @@ extern "C" int focus_lm_head_conf_noalloc(const float* hidden, int32_t rows, int
         !(rms_eps >= 0.f))
         return FOCUS_ERR_INVALID_ARG;
     if (rows > kNaRows || hidden_dim > kNaDim || vocab > kNaVocab) return FOCUS_ERR_LIMITS;
-    if (hidden_dim % BK) return FOCUS_ERR_UNSUPPORTED;
+    if (hidden_dim % 128) return FOCUS_ERR_UNSUPPORTED;
     if (rows == 0) return FOCUS_OK;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return FOCUS_ERR_CUDA;
@@ -145,7 +144,7 @@ extern "C" int focus_lm_head_conf_noalloc(const float* hidden, int32_t rows, int
         return FOCUS_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(flag, 0, sizeof(int), s) != cudaSuccess) return FOCUS_ERR_CUDA;
-    na_norm_kernel<<<rows, 256, 0, s>>>(hidden, hidden_dim, static_cast<const bf16*>(final_norm), rms_eps, h);
+    na_norm_kernel<<<rows, kNormThreads, 0, s>>>(hidden, hidden_dim, static_cast<const bf16*>(final_norm), rms_eps, h);
     GemmArgs g{};
     g.A = h;
     g.B = lm_head;

@@ -1,6 +1,8 @@
 // Row-wise kernels of the step: embedding + RMSNorm, residual reduction + RMSNorm (optionally
 // gathering the kept rows), and the QKV finalisation (RoPE + intra-block KV-cache write).
-// All three are HBM-bound row sweeps: one CTA per row, coalesced loads, fixed-order reductions.
+// With a few dozen kept rows these kernels are latency-bound, so each CTA takes one row and issues
+// every load of the row (float4, all in flight together) before using any; reductions run in a fixed
+// order.
 #include "launch.h"
 
 namespace focus {
@@ -8,57 +10,85 @@ namespace focus {
 namespace {
 
 constexpr int kRowThreads = 256;
+constexpr int kMaxNormSplits = 8;  // split-K partial slices a norm kernel adds (CUDA-core path: at most 1)
 
+// One CTA per row: x = E[token], h = RMSNorm(x) * gamma.
 template <typename T>
-__global__ void __launch_bounds__(kRowThreads) embed_norm_kernel(const int32_t* __restrict__ tokens, int V,
-                                                                 const T* __restrict__ embed,
-                                                                 const T* __restrict__ gamma, float eps, int D,
-                                                                 float* __restrict__ x, T* __restrict__ h,
-                                                                 int* err) {
+__global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(const int32_t* __restrict__ tokens, int V,
+                                                                  const T* __restrict__ embed,
+                                                                  const T* __restrict__ gamma, float eps, int D,
+                                                                  float* __restrict__ x, T* __restrict__ h, int* err) {
     __shared__ float red[32];
-    const int r = blockIdx.x;
+    const int r = blockIdx.x, tid = threadIdx.x;
     int tok = tokens[r];
     if (tok < 0 || tok >= V) {
-        if (threadIdx.x == 0) raise_err(err, FOCUS_DEVERR_TOKEN_ID);
+        if (tid == 0) raise_err(err, FOCUS_DEVERR_TOKEN_ID);
         tok = 0;
     }
     const T* e = embed + (size_t)tok * D;
     float* xr = x + (size_t)r * D;
-    float ss = 0.f;
-    for (int i = threadIdx.x; i < D; i += blockDim.x) {
-        float v = to_f(e[i]);
-        xr[i] = v;
-        ss += v * v;
+    float4 v[kNormVec];
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+        const int c = (i * kNormThreads + tid) * 4;
+        v[i] = c < D ? load4<T>(e + c) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const float tot = block_sum(ss, red);
-    const float inv = rsqrtf(tot / D + eps);
-    T* hr = h + (size_t)r * D;
-    for (int i = threadIdx.x; i < D; i += blockDim.x) hr[i] = from_f<T>(xr[i] * inv * to_f(gamma[i]));
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+        const int c = (i * kNormThreads + tid) * 4;
+        if (c < D) *reinterpret_cast<float4*>(xr + c) = v[i];
+    }
+    rmsnorm_finish_cta<T>(v, D, gamma, eps, h + (size_t)r * D, red);
 }
 
+// One CTA per row: x_out[r] = x_in[src] + the split partials (src = src_map ? src_map[r] : r), then
+// h_out[r] = RMSNorm(x_out[r]) * gamma.  Every load of the row is issued before any is used.
 template <typename T>
-__global__ void __launch_bounds__(kRowThreads) residual_norm_kernel(
+__global__ void __launch_bounds__(kNormThreads) residual_norm_kernel(
     const float* __restrict__ x_in, const int32_t* __restrict__ src_map, const int32_t* __restrict__ n_rows_dev,
     const float* __restrict__ part, int n_splits, size_t part_stride, float* x_out, const T* __restrict__ gamma,
     float eps, int D, T* __restrict__ h_out) {
     __shared__ float red[32];
-    const int r = blockIdx.x;
+    const int r = blockIdx.x, tid = threadIdx.x;
     if (n_rows_dev && r >= *n_rows_dev) return;
     const int src = src_map ? src_map[r] : r;
     const float* xi = x_in + (size_t)src * D;
     float* xo = x_out + (size_t)r * D;
-    float ss = 0.f;
-    for (int i = threadIdx.x; i < D; i += blockDim.x) {
-        float v = xi[i];
-        for (int s = 0; s < n_splits; ++s) v += part[(size_t)s * part_stride + (size_t)src * D + i];
-        xo[i] = v;
-        ss += v * v;
+    float4 v[kNormVec];
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+        const int c = (i * kNormThreads + tid) * 4;
+        v[i] = c < D ? *reinterpret_cast<const float4*>(xi + c) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (!h_out) return;
-    const float tot = block_sum(ss, red);
-    const float inv = rsqrtf(tot / D + eps);
-    T* hr = h_out + (size_t)r * D;
-    for (int i = threadIdx.x; i < D; i += blockDim.x) hr[i] = from_f<T>(xo[i] * inv * to_f(gamma[i]));
+    if (n_splits > 0) {
+        float4 p[kNormVec][kMaxNormSplits];
+#pragma unroll
+        for (int i = 0; i < kNormVec; ++i)
+#pragma unroll
+            for (int sp = 0; sp < kMaxNormSplits; ++sp) {
+                const int c = (i * kNormThreads + tid) * 4;
+                p[i][sp] = (c < D && sp < n_splits)
+                               ? *reinterpret_cast<const float4*>(part + (size_t)sp * part_stride + (size_t)src * D + c)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+        for (int i = 0; i < kNormVec; ++i)
+#pragma unroll
+            for (int sp = 0; sp < kMaxNormSplits; ++sp) {
+                v[i].x += p[i][sp].x;
+                v[i].y += p[i][sp].y;
+                v[i].z += p[i][sp].z;
+                v[i].w += p[i][sp].w;
+            }
+    }
+    if (n_splits > 0 || xo != xi) {  // in-place normalisation alone leaves x untouched
+#pragma unroll
+        for (int i = 0; i < kNormVec; ++i) {
+            const int c = (i * kNormThreads + tid) * 4;
+            if (c < D) *reinterpret_cast<float4*>(xo + c) = v[i];
+        }
+    }
+    if (h_out) rmsnorm_finish_cta<T>(v, D, gamma, eps, h_out + (size_t)r * D, red);
 }
 
 template <typename T>
@@ -77,10 +107,14 @@ __global__ void __launch_bounds__(kRowThreads) qkv_finalize_kernel(const float* 
     const int P = checked_prefix(prefix_len, b, max_prefix, err);
     const double pos = (double)(P + j);
     for (int i = threadIdx.x; i < half; i += blockDim.x) {
-        double sn, cn;
-        sincos(pos * inv_freq[i], &sn, &cn);
-        cs[i] = (float)cn;
-        cs[half + i] = (float)sn;
+        // angle reduced to [-pi, pi] in double (two-term 2*pi, Cody-Waite), then a float sincos
+        const double ang = pos * inv_freq[i];
+        const double k = rint(ang * 0.15915494309189535);
+        const double red = (ang - k * 6.283185307179586) - k * 2.4492935982947064e-16;
+        float sn, cn;
+        sincosf((float)red, &sn, &cn);
+        cs[i] = cn;
+        cs[half + i] = sn;
     }
     __syncthreads();
     const int B = rm.block;
@@ -123,7 +157,7 @@ template <typename T>
 int launch_embed_norm(const int32_t* tokens, int rows, int V, const T* embed, const T* gamma, float eps, int D,
                        float* x, T* h, int* err, cudaStream_t s) {
     if (rows <= 0) return 0;
-    embed_norm_kernel<T><<<rows, kRowThreads, 0, s>>>(tokens, V, embed, gamma, eps, D, x, h, err);
+    embed_norm_kernel<T><<<rows, kNormThreads, 0, s>>>(tokens, V, embed, gamma, eps, D, x, h, err);
     return 1;
 }
 
@@ -132,8 +166,8 @@ int launch_residual_norm(const float* x_in, const int32_t* src_map, const int32_
                           const float* part, int n_splits, size_t part_stride, float* x_out, const T* gamma,
                           float eps, int D, T* h_out, cudaStream_t s) {
     if (rows_bound <= 0) return 0;
-    residual_norm_kernel<T><<<rows_bound, kRowThreads, 0, s>>>(x_in, src_map, n_rows_dev, part, n_splits,
-                                                               part_stride, x_out, gamma, eps, D, h_out);
+    residual_norm_kernel<T><<<rows_bound, kNormThreads, 0, s>>>(x_in, src_map, n_rows_dev, part, n_splits, part_stride,
+                                                                x_out, gamma, eps, D, h_out);
     return 1;
 }
 
@@ -145,6 +179,15 @@ int launch_qkv_finalize(const float* part, int n_splits, size_t part_stride, Row
     qkv_finalize_kernel<T><<<rm.rows_static, kRowThreads, dm.d * sizeof(float), s>>>(
         part, n_splits, part_stride, rm, prefix_len, max_prefix, inv_freq, dm, layer, q_out, ibc, err);
     return 1;
+}
+
+bool configure_rows_kernels() {
+    return max_shared_carveout((const void*)embed_norm_kernel<float>) &&
+           max_shared_carveout((const void*)embed_norm_kernel<bf16>) &&
+           max_shared_carveout((const void*)residual_norm_kernel<float>) &&
+           max_shared_carveout((const void*)residual_norm_kernel<bf16>) &&
+           max_shared_carveout((const void*)qkv_finalize_kernel<float>) &&
+           max_shared_carveout((const void*)qkv_finalize_kernel<bf16>);
 }
 
 #define FOCUS_INST_ROWS(T)                                                                                         \

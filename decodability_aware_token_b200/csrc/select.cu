@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(1024) select_kernel(SelectArgs a) {
             msk[h] = false;
             if (valid[h]) {
                 float i0 = 0.f, i1 = 0.f;
+#pragma unroll 8
                 for (int g = 0; g < a.groups; ++g) {  // partial groups in order: deterministic
                     i0 += a.imp_part[((size_t)b * a.groups + g) * B + j];
                     i1 += a.imp_part[layer_stride + ((size_t)b * a.groups + g) * B + j];
@@ -140,6 +141,8 @@ __global__ void __launch_bounds__(1024) select_kernel(SelectArgs a) {
 }
 
 }  // namespace
+
+bool configure_select_kernel() { return max_shared_carveout((const void*)select_kernel); }
 
 int launch_select(const SelectArgs& a, cudaStream_t s) {
     if (a.N <= 0) return 0;

@@ -23,8 +23,16 @@ namespace {
 using namespace tc;
 
 // ------------------------------------------------------------------ host side
-constexpr int kBN = 128, kMSUB = 2, kStages = 4;
-using Shape = TcShape<kBN, kMSUB, kStages>;
+// Two tile configurations.  Many rows (layers 0-1: N*B rows): 256 x 128 tiles, two 128-row TMEM
+// accumulators sharing each weight tile.  Few rows (layers 2..L-1 and the LM head: at most N*k_max
+// kept rows, typically a few dozen): 128-row tiles, CTAs whose rows are all beyond the live row count
+// exit at once, so no MMA work or activation traffic is spent on absent rows; SwiGLU uses 64-wide
+// tiles (32 gate + 32 up columns) so that twice as many CTAs stream the gate / up weights.
+constexpr int kBN = 128, kStages = 4;
+constexpr int kSmallRows = 256;  // GEMMs with at most this many rows use the few-rows tiles
+using Big = TcShape<kBN, 2, kStages>;
+using Small = TcShape<kBN, 1, kStages>;
+using SmallGlu = TcShape<64, 1, kStages>;
 
 }  // namespace
 
@@ -32,10 +40,14 @@ struct TcPlan {
     Dims dm;
     int rows_full, rows_c;
     const void *h, *o, *act;
-    CUtensorMap map_h, map_o, map_act;
-    std::unordered_map<const void*, CUtensorMap> wmap;  // weight pointer -> tensor map
+    CUtensorMap map_h, map_o, map_act;        // 256-row boxes
+    CUtensorMap map_h1, map_o1, map_act1;     // 128-row boxes
+    std::unordered_map<const void*, CUtensorMap> wmap;   // weight pointer -> map (box rows = tile N or N/2)
+    std::unordered_map<const void*, CUtensorMap> wmap1;  // gate / up maps for the 64-wide SwiGLU tile
     int* err;
 };
+
+
 
 int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, void* o, void* act, int rows_full,
                    int rows_c, int lm_tiles_cap, int* err) {
@@ -52,19 +64,25 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
     p->o = o;
     p->act = act;
     p->err = err;
-    bool ok = make_map(&p->map_h, h, rows_full, dm.D, Shape::BM) &&
-              make_map(&p->map_o, o, rows_full, (uint64_t)dm.Hq * dm.d, Shape::BM) &&
-              make_map(&p->map_act, act, rows_full, dm.F, Shape::BM);
+    const uint64_t HD = (uint64_t)dm.Hq * dm.d;
+    bool ok = make_map(&p->map_h, h, rows_full, dm.D, Big::BM) && make_map(&p->map_o, o, rows_full, HD, Big::BM) &&
+              make_map(&p->map_act, act, rows_full, dm.F, Big::BM) &&
+              make_map(&p->map_h1, h, rows_full, dm.D, Small::BM) && make_map(&p->map_o1, o, rows_full, HD, Small::BM) &&
+              make_map(&p->map_act1, act, rows_full, dm.F, Small::BM);
     for (int l = 0; ok && l < w.L; ++l) {
         CUtensorMap m;
         ok = ok && make_map(&m, w.wqkv[l], dm.qkv, dm.D, kBN);
         p->wmap[w.wqkv[l]] = m;
-        ok = ok && make_map(&m, w.wo[l], dm.D, (uint64_t)dm.Hq * dm.d, kBN);
+        ok = ok && make_map(&m, w.wo[l], dm.D, HD, kBN);
         p->wmap[w.wo[l]] = m;
         ok = ok && make_map(&m, w.wgate[l], dm.F, dm.D, kBN / 2);
         p->wmap[w.wgate[l]] = m;
         ok = ok && make_map(&m, w.wup[l], dm.F, dm.D, kBN / 2);
         p->wmap[w.wup[l]] = m;
+        ok = ok && make_map(&m, w.wgate[l], dm.F, dm.D, 32);
+        p->wmap1[w.wgate[l]] = m;
+        ok = ok && make_map(&m, w.wup[l], dm.F, dm.D, 32);
+        p->wmap1[w.wup[l]] = m;
         ok = ok && make_map(&m, w.wdown[l], dm.D, dm.F, kBN);
         p->wmap[w.wdown[l]] = m;
     }
@@ -75,12 +93,20 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
         delete p;
         return FOCUS_ERR_CUDA;
     }
-    auto set_smem = [](const void* fn) {
-        return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, Shape::SMEM) == cudaSuccess;
+    auto set_smem = [](const void* fn, int bytes) {
+        return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
+               max_shared_carveout(fn);
     };
-    ok = set_smem((const void*)tc_gemm_kernel<kBN, kMSUB, kStages, EPI_PARTIAL>) &&
-         set_smem((const void*)tc_gemm_kernel<kBN, kMSUB, kStages, EPI_SWIGLU>) &&
-         set_smem((const void*)tc_gemm_kernel<kBN, kMSUB, kStages, EPI_LMHEAD>);
+    ok = set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_PARTIAL>, Big::SMEM) &&
+         set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_SWIGLU>, Big::SMEM) &&
+         set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_LMHEAD>, Big::SMEM) &&
+         set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_RESID>, Big::SMEM) &&
+         set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_QKV>, Big::SMEM) &&
+         set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL>, Small::SMEM) &&
+         set_smem((const void*)tc_gemm_kernel<64, 1, kStages, EPI_SWIGLU>, SmallGlu::SMEM) &&
+         set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_LMHEAD>, Small::SMEM) &&
+         set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_RESID>, Small::SMEM) &&
+         set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_QKV>, Small::SMEM);
     if (!ok) {
         delete p;
         return FOCUS_ERR_CUDA;
@@ -92,7 +118,9 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
 void tc_plan_destroy(TcPlan* p) { delete p; }
 
 int tc_splits(const TcPlan* p, int wid, int m_bound) {
-    if (!p || m_bound > Shape::BM) return 1;  // only single-M-tile GEMMs split K
+    // few-row GEMMs split K so that about 128 CTAs stream each weight matrix; the split partials are
+    // reduced inside the GEMM by the last CTA of each output tile (at most kMaxReduceSplits of them)
+    if (!p || m_bound > kSmallRows) return 1;
     switch (wid) {
         case W_QKV: return 4;
         case W_O: return 8;
@@ -106,31 +134,65 @@ int tc_lm_tiles(const TcPlan* p) { return p ? (p->dm.V + kBN - 1) / kBN : 0; }
 int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g0, cudaStream_t s) {
     if (g0.M_bound <= 0) return 0;
     GemmArgs g = g0;
-    const CUtensorMap* a = g.A == p->h ? &p->map_h : g.A == p->o ? &p->map_o : &p->map_act;
-    auto itb = p->wmap.find(g.B);
-    const CUtensorMap* b = &itb->second;
+    const bool small = g.M_bound <= kSmallRows;
+    const CUtensorMap* a = g.A == p->h ? (small ? &p->map_h1 : &p->map_h)
+                         : g.A == p->o ? (small ? &p->map_o1 : &p->map_o)
+                                       : (small ? &p->map_act1 : &p->map_act);
+    const CUtensorMap* b = &p->wmap.find(g.B)->second;
     const CUtensorMap* b2 = b;
-    if (epi == EPI_SWIGLU) b2 = &p->wmap.find(g.B2)->second;
-    int splits = epi == EPI_PARTIAL ? g.splits : 1;
+    if (epi == EPI_SWIGLU) {
+        auto& wm = small ? p->wmap1 : p->wmap;
+        b = &wm.find(g.B)->second;
+        b2 = &wm.find(g.B2)->second;
+    }
+    int splits = (epi == EPI_PARTIAL || epi == EPI_RESID || epi == EPI_QKV) ? g.splits : 1;
     if (splits > g.K / BK) splits = g.K / BK;  // every split slice gets at least one K block
     if (splits < 1) splits = 1;
-    const int n_tiles = epi == EPI_SWIGLU ? g.N / (kBN / 2) : (g.N + kBN - 1) / kBN;
+    const int glu_cols = small ? 32 : kBN / 2;  // output columns per SwiGLU tile
+    const int n_tiles = epi == EPI_SWIGLU ? g.N / glu_cols : (g.N + kBN - 1) / kBN;
     if (epi == EPI_LMHEAD) {
         g.n_tiles = n_tiles;
         g.tile_n = kBN;
     }
-    dim3 grid(n_tiles, (g.M_bound + Shape::BM - 1) / Shape::BM, splits);
+    const int bm = small ? Small::BM : Big::BM;
+    dim3 grid(n_tiles, (g.M_bound + bm - 1) / bm, splits);
     (void)wid;
-    switch (epi) {
-        case EPI_PARTIAL:
-            tc_gemm_kernel<kBN, kMSUB, kStages, EPI_PARTIAL><<<grid, 192, Shape::SMEM, s>>>(*a, *b, *b2, g, p->err);
-            break;
-        case EPI_SWIGLU:
-            tc_gemm_kernel<kBN, kMSUB, kStages, EPI_SWIGLU><<<grid, 192, Shape::SMEM, s>>>(*a, *b, *b2, g, p->err);
-            break;
-        case EPI_LMHEAD:
-            tc_gemm_kernel<kBN, kMSUB, kStages, EPI_LMHEAD><<<grid, 192, Shape::SMEM, s>>>(*a, *b, *b2, g, p->err);
-            break;
+    if (small) {
+        switch (epi) {
+            case EPI_PARTIAL:
+                tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
+                break;
+            case EPI_SWIGLU:
+                tc_gemm_kernel<64, 1, kStages, EPI_SWIGLU><<<grid, 192, SmallGlu::SMEM, s>>>(*a, *b, *b2, g, p->err);
+                break;
+            case EPI_LMHEAD:
+                tc_gemm_kernel<kBN, 1, kStages, EPI_LMHEAD><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
+                break;
+            case EPI_RESID:
+                tc_gemm_kernel<kBN, 1, kStages, EPI_RESID><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
+                break;
+            case EPI_QKV:
+                tc_gemm_kernel<kBN, 1, kStages, EPI_QKV><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
+                break;
+        }
+    } else {
+        switch (epi) {
+            case EPI_PARTIAL:
+                tc_gemm_kernel<kBN, 2, kStages, EPI_PARTIAL><<<grid, 192, Big::SMEM, s>>>(*a, *b, *b2, g, p->err);
+                break;
+            case EPI_SWIGLU:
+                tc_gemm_kernel<kBN, 2, kStages, EPI_SWIGLU><<<grid, 192, Big::SMEM, s>>>(*a, *b, *b2, g, p->err);
+                break;
+            case EPI_LMHEAD:
+                tc_gemm_kernel<kBN, 2, kStages, EPI_LMHEAD><<<grid, 192, Big::SMEM, s>>>(*a, *b, *b2, g, p->err);
+                break;
+            case EPI_RESID:
+                tc_gemm_kernel<kBN, 2, kStages, EPI_RESID><<<grid, 192, Big::SMEM, s>>>(*a, *b, *b2, g, p->err);
+                break;
+            case EPI_QKV:
+                tc_gemm_kernel<kBN, 2, kStages, EPI_QKV><<<grid, 192, Big::SMEM, s>>>(*a, *b, *b2, g, p->err);
+                break;
+        }
     }
     return 1;
 }

@@ -112,6 +112,40 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// RoPE angle of block position pos for pair i: reduced modulo 2 pi in double (two-term 2 pi), then a
+// float sincos on [-pi, pi].
+__device__ __forceinline__ void rope_cs(int pos, double inv_freq, float& cn, float& sn) {
+    const double ang = (double)pos * inv_freq;
+    const double k = rint(ang * 0.15915494309189535);
+    const double red = (ang - k * 6.283185307179586) - k * 2.4492935982947064e-16;
+    sincosf((float)red, &sn, &cn);
+}
+
+// (request, block position, rotary position) of a GEMM row in the QKV epilogue
+__device__ __forceinline__ void qkv_row(const GemmArgs& g, int row, int& b, int& j, int& pos) {
+    if (g.row_req) {
+        b = g.row_req[row];
+        j = g.row_pos[row];
+    } else {
+        b = row / g.block;
+        j = row - b * g.block;
+    }
+    pos = checked_prefix(g.prefix_len, b, g.max_prefix, g.err) + j;
+}
+
+// destination of 128-wide head tile `head` of a QKV row: query rows, or K / V of the intra-block cache
+__device__ __forceinline__ bf16* qkv_dst(const GemmArgs& g, int row, int head, int b, int j) {
+    if (head < g.Hq) return reinterpret_cast<bf16*>(g.q_out) + ((size_t)row * g.Hq + head) * 128;
+    const int kv = head < g.Hq + g.Hkv ? 0 : 1;
+    const int gh = head - g.Hq - kv * g.Hkv;
+    return reinterpret_cast<bf16*>(g.ibc) +
+           ((((size_t)b * g.n_layers + g.layer) * 2 + kv) * g.Hkv + gh) * (size_t)g.block * 128 + (size_t)j * 128;
+}
+
+__device__ __forceinline__ void named_sync_epilogue() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+constexpr int kMaxReduceSplits = 8;  // split-K slices the fused reduction sums (the launcher never uses more)
+
 template <int BN, int MSUB, int STAGES>
 struct TcShape {
     static constexpr int BM = 128 * MSUB;
@@ -246,6 +280,71 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
                         for (int q = 0; q < 8; ++q) o4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                     }
                 }
+            } else if (EPI == EPI_RESID || EPI == EPI_QKV) {
+                if (gridDim.z > 1) {
+                    // split K: leave this split's partial tile; the tile's last CTA reduces below
+                    float* out = g.part + (size_t)split * g.split_stride + (size_t)row * g.N + (size_t)n_tile * BN;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < BN; c0 += 32) {
+                        float v[32];
+                        tmem_ld32(tbase + c0, v);
+                        if (live) {
+                            float4* o4 = reinterpret_cast<float4*>(out + c0);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                o4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                        }
+                    }
+                } else if (EPI == EPI_RESID) {
+                    float* xr = g.resid + (size_t)row * g.N + (size_t)n_tile * BN;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < BN; c0 += 32) {
+                        float v[32];
+                        tmem_ld32(tbase + c0, v);
+                        if (live) {
+                            float4* x4 = reinterpret_cast<float4*>(xr + c0);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                float4 x = x4[q];
+                                x.x += v[4 * q];
+                                x.y += v[4 * q + 1];
+                                x.z += v[4 * q + 2];
+                                x.w += v[4 * q + 3];
+                                x4[q] = x;
+                            }
+                        }
+                    }
+                } else {
+                    // one head per 128-column tile: rotate pairs (i, i + 64), then q rows or the cache
+                    const int head = n_tile;
+                    const bool rotate = head < g.Hq + g.Hkv;
+                    int b = 0, j = 0, pos = 0;
+                    if (live) qkv_row(g, row, b, j, pos);
+#pragma unroll 1
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
+                        float lo[32], hi[32];
+                        tmem_ld32(tbase + c0, lo);
+                        tmem_ld32(tbase + 64 + c0, hi);
+                        if (live) {
+                            bf16* dst = qkv_dst(g, row, head, b, j);
+#pragma unroll
+                            for (int t = 0; t < 32; t += 2) {
+                                float a0 = lo[t], a1 = lo[t + 1], b0 = hi[t], b1 = hi[t + 1];
+                                if (rotate) {
+                                    float c_0, s_0, c_1, s_1;
+                                    rope_cs(pos, g.inv_freq[c0 + t], c_0, s_0);
+                                    rope_cs(pos, g.inv_freq[c0 + t + 1], c_1, s_1);
+                                    a0 = lo[t] * c_0 - hi[t] * s_0;
+                                    b0 = hi[t] * c_0 + lo[t] * s_0;
+                                    a1 = lo[t + 1] * c_1 - hi[t + 1] * s_1;
+                                    b1 = hi[t + 1] * c_1 + lo[t + 1] * s_1;
+                                }
+                                *reinterpret_cast<__nv_bfloat162*>(dst + c0 + t) = __floats2bfloat162_rn(a0, a1);
+                                *reinterpret_cast<__nv_bfloat162*>(dst + 64 + c0 + t) = __floats2bfloat162_rn(b0, b1);
+                            }
+                        }
+                    }
+                }
             } else if (EPI == EPI_SWIGLU) {
                 bf16* out = reinterpret_cast<bf16*>(g.act) + (size_t)row * g.N + (size_t)n_tile * (BN / 2);
 #pragma unroll 1
@@ -306,6 +405,83 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
                     g.lm_max[idx] = mx;
                     g.lm_sum[idx] = se;
                     g.lm_arg[idx] = arg;
+                }
+            }
+        }
+        if constexpr (EPI == EPI_RESID || EPI == EPI_QKV) {
+            if (gridDim.z > 1) {  // block-uniform: every epilogue thread reaches both barriers
+                // last split CTA of this output tile: sum the splits in order and apply the epilogue
+                // (a split that timed out still counts its arrival; its outputs are flagged invalid)
+                __shared__ int last_split;
+                __threadfence();
+                named_sync_epilogue();
+                const int tile_id = blockIdx.y * gridDim.x + blockIdx.x;
+                if (warp == 2 && lane == 0) last_split = atomicAdd(&g.counters[tile_id], 1) == (int)gridDim.z - 1;
+                named_sync_epilogue();
+                if (last_split) {
+                    __threadfence();
+                    const int ew = warp - 2;
+                    const int col = lane * 4;  // BN == 128: 32 lanes x 4 columns
+                    const int rmax = M < m0 + S::BM ? M : m0 + S::BM;
+                    const int nsp = (int)gridDim.z;
+                    // 4 rows per pass, every split of them loaded before any is summed (one L2 round trip),
+                    // then summed in split order
+                    for (int r0 = m0 + ew; r0 < rmax; r0 += 16) {
+                        float4 pv[4][kMaxReduceSplits];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+#pragma unroll
+                            for (int sp = 0; sp < kMaxReduceSplits; ++sp)
+                                pv[q][sp] = (sp < nsp && r0 + 4 * q < rmax)
+                                                ? __ldcg(reinterpret_cast<const float4*>(
+                                                      g.part + (size_t)sp * g.split_stride +
+                                                      (size_t)(r0 + 4 * q) * g.N + (size_t)n_tile * BN + col))
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int row = r0 + 4 * q;
+                        if (row >= rmax) continue;  // warp-uniform (the row depends on the warp only)
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                        for (int sp = 0; sp < kMaxReduceSplits; ++sp) {
+                            acc.x += pv[q][sp].x;
+                            acc.y += pv[q][sp].y;
+                            acc.z += pv[q][sp].z;
+                            acc.w += pv[q][sp].w;
+                        }
+                        if (EPI == EPI_RESID) {
+                            float4* x4 = reinterpret_cast<float4*>(g.resid + (size_t)row * g.N + (size_t)n_tile * BN + col);
+                            float4 x = *x4;
+                            x.x += acc.x;
+                            x.y += acc.y;
+                            x.z += acc.z;
+                            x.w += acc.w;
+                            *x4 = x;
+                        } else {
+                            const int head = n_tile;
+                            int b, j, pos;
+                            qkv_row(g, row, b, j, pos);
+                            float v[4] = {acc.x, acc.y, acc.z, acc.w};
+                            float o4[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float partner = __shfl_xor_sync(0xffffffffu, v[e], 16);  // column +- 64
+                                if (head < g.Hq + g.Hkv) {
+                                    const int i = (col + e) & 63;
+                                    float cn, sn;
+                                    rope_cs(pos, g.inv_freq[i], cn, sn);
+                                    o4[e] = col < 64 ? v[e] * cn - partner * sn : v[e] * cn + partner * sn;
+                                } else {
+                                    o4[e] = v[e];
+                                }
+                            }
+                            bf16* dst = qkv_dst(g, row, head, b, j) + col;
+                            *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(o4[0], o4[1]);
+                            *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __floats2bfloat162_rn(o4[2], o4[3]);
+                        }
+                    }
+                    }
+                    if (warp == 2 && lane == 0) g.counters[tile_id] = 0;  // ready for the next launch
                 }
             }
         }

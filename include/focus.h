@@ -125,7 +125,7 @@ typedef struct {
 typedef struct {
     int32_t n_requests;          /* N */
     int32_t block_size;          /* B */
-    int32_t page_size;           /* S: tokens per KV page */
+    int32_t page_size;           /* S: tokens per KV page (bf16 models: 16, 32 or 64) */
     int32_t n_pages;             /* number of pages in kv_pool */
     int32_t* block_tokens;       /* [N, B] int32, updated in place: decoded positions get their id */
     uint8_t* mask;               /* [N, B] uint8, nonzero = still masked; updated in place (decoded -> 0) */
@@ -165,7 +165,7 @@ typedef struct focus_ctx focus_ctx;
 /* Validate the model and limits, record the (borrowed) weight pointers, allocate
  * the workspace and build the TMA descriptors of every weight matrix.  Uses the
  * current CUDA device.  Supported: L >= 2, Hq % Hkv == 0, d in {64, 128} (128 for
- * bf16), D % 64 == 0, F % 64 == 0, B <= 64, max_keep <= max_block.
+ * bf16), D % 128 == 0, F % 64 == 0, B <= 64, max_keep <= max_block.
  * Returns FOCUS_OK and *out, or an error with *out = NULL. */
 int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_limits* lim, focus_ctx** out);
 
@@ -218,7 +218,9 @@ int focus_last_step_launches(const focus_ctx* ctx);
 
 /* From now on, record a CUDA event pair (on the step's stream) around every launch of
  * `kernel_class` in later focus_step calls, for at most `max_launches` launches.  Host-side only;
- * costs two event records per timed launch.  Returns FOCUS_ERR_INVALID_ARG on a bad class. */
+ * costs two event records per timed launch.  A step captured into a CUDA graph while recording keeps
+ * the pairs as event nodes: focus_profile_end then reports the most recent replay.  Returns
+ * FOCUS_ERR_INVALID_ARG on a bad class. */
 int focus_profile_begin(focus_ctx* ctx, int kernel_class, int max_launches);
 
 /* Stop recording, synchronise the device, and return the summed device time of the recorded
@@ -239,8 +241,8 @@ int focus_profile_end(focus_ctx* ctx, float* total_ms, int32_t* launches);
  *   conf        [rows] float32, device (out); top_id [rows] int32, device (out)
  *   stream      cudaStream_t (NULL = legacy default stream); the call is asynchronous
  *
- * Limits: rows <= 256, hidden_dim <= 4096 and a multiple of 64, vocab <= 163840; larger sizes return
- * FOCUS_ERR_LIMITS (FOCUS_ERR_UNSUPPORTED for a hidden_dim that is not a multiple of 64) and launch
+ * Limits: rows <= 256, hidden_dim <= 4096 and a multiple of 128, vocab <= 163840; larger sizes return
+ * FOCUS_ERR_LIMITS (FOCUS_ERR_UNSUPPORTED for a hidden_dim that is not a multiple of 128) and launch
  * nothing.  rows == 0 returns FOCUS_OK at once.  The first call on a device looks up the array's
  * device address (with that device current) and must therefore come before any stream capture on
  * that device.  All calls on a device share the array: calls that may overlap on the GPU race on it

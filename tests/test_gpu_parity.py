@@ -169,6 +169,38 @@ def test_step_is_deterministic():
     assert torch.equal(a["ibc"], b["ibc"])
 
 
+def test_step_replays_from_cuda_graph():
+    """focus_step makes no host synchronisation: a captured step replays with the eager step's results."""
+    from decodability_aware_token_b200 import FocusContext, StepParams
+    case = _case("small_bf16")
+    w = case.work
+    m = _model("small_bf16", case)
+    lim = limits_for(case, step_params(w))
+    dev = torch.device("cuda:0")
+    batch = {k: v.to(dev).clone() for k, v in case.batch.items()}
+    tok0, mask0 = batch["block_tokens"].clone(), batch["mask"].clone()
+    p = StepParams(w.tau, w.k_min, w.k_max, w.conf_threshold)
+    with FocusContext(case.shape, m, **lim) as ctx:
+        eager = ctx.step(batch, p)
+        torch.cuda.synchronize()
+        ref = {k: v.clone() for k, v in eager.tensors().items() if v is not None}
+        ref_ibc = batch["ibc"].clone()
+        out = ctx.alloc_outputs(w.n_requests, w.block)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            batch["block_tokens"].copy_(tok0)
+            batch["mask"].copy_(mask0)
+            ctx.step(batch, p, out)
+        for _ in range(2):
+            g.replay()
+            torch.cuda.synchronize()
+            for k, v in ref.items():
+                assert torch.equal(getattr(out, k), v), k
+            assert torch.equal(batch["ibc"], ref_ibc)
+        rc, bits = ctx.device_error()
+        assert rc == 0, bits
+
+
 # ---------------------------------------------------------------- full-size workloads, sampled requests
 @pytest.mark.slow
 def test_sdar_1p7b_n32_b32_sampled():
