@@ -55,7 +55,6 @@ struct focus_ctx {
 namespace {
 
 constexpr int kMaxSplits = 8;
-constexpr int kGemmCounters = 1024;  // output tiles of one split-K GEMM launch (at most 2 x 48 here)
 
 struct Layout {
     size_t off[32];
@@ -284,9 +283,8 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
                                        W(g_next), dm.eps, dm.D, h, s);
     });
     // ---- layers 2..L-1 on the kept rows
-    const int sp_qkv = tc ? tc_splits(c->tc, W_QKV, R_bound) : 1;
-    const int sp_o = tc ? tc_splits(c->tc, W_O, R_bound) : 1;
-    const int sp_dn = tc ? tc_splits(c->tc, W_DOWN, R_bound) : 1;
+    // the tensor-core GEMMs pick their own split-K for the kept rows and reduce it in the epilogue
+    const int sp_qkv = 1, sp_o = 1, sp_dn = 1;
     for (int l = 2; l < dm.L; ++l) {
         if (tc) {
             gemm(FOCUS_K_GEMM_QKV, EPI_QKV, c->h, c->wqkv[l], nullptr, R_bound, c->n_rows, dm.qkv, dm.D, sp_qkv, W_QKV,

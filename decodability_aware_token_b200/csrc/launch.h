@@ -133,6 +133,7 @@ struct GemmArgs {
     int* err;
 };
 template <typename T> int launch_gemm_simt(Epi epi, const GemmArgs& g, cudaStream_t s);
+constexpr int kGemmCounters = 1024;  // arrival counters: output tiles of one split-K GEMM launch
 constexpr int kSimtTileN = 64;
 
 // ---- LM-head combine + threshold decode (decode.cu) ------------------------------

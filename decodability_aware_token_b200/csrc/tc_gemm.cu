@@ -3,6 +3,11 @@
 //   EPI_PARTIAL: float32 partial sums of one split-K slice -> part[split][m][n]
 //   EPI_SWIGLU:  the B tile is BN/2 gate rows followed by BN/2 up rows; writes silu(g) * u (bf16)
 //   EPI_LMHEAD:  per row and vocabulary tile: max logit, sum exp(z - max), first argmax (no logits in HBM)
+//   EPI_RESID:   resid += A B^T (float32 residual stream)
+//   EPI_QKV:     rotary embedding of the query / key heads, queries to q, keys and values to the cache
+//
+// GEMMs of at most 256 rows with the RESID, QKV or SWIGLU epilogue run on the swapped kernel
+// (features on the MMA's M side, tokens on N); the rest on the row-major kernel below.
 //
 // One CTA computes a (128 * MSUB) x BN tile (MSUB accumulators of 128 x BN fp32 in TMEM) over a range of
 // 64-wide K blocks.  Warp roles: warp 0 lane 0 issues TMA loads into a STAGES-deep shared-memory ring,
@@ -23,16 +28,14 @@ namespace {
 using namespace tc;
 
 // ------------------------------------------------------------------ host side
-// Two tile configurations.  Many rows (layers 0-1: N*B rows): 256 x 128 tiles, two 128-row TMEM
-// accumulators sharing each weight tile.  Few rows (layers 2..L-1 and the LM head: at most N*k_max
-// kept rows, typically a few dozen): 128-row tiles, CTAs whose rows are all beyond the live row count
-// exit at once, so no MMA work or activation traffic is spent on absent rows; SwiGLU uses 64-wide
-// tiles (32 gate + 32 up columns) so that twice as many CTAs stream the gate / up weights.
+// Many rows (layers 0-1: N*B rows): 256 x 128 tiles, two 128-row TMEM accumulators sharing each weight
+// tile.  Few rows (layers 2..L-1 and the LM head: at most N*k_max kept rows, typically a few dozen):
+// the swapped kernel for QKV / O / gate-up / down, and 128-row tiles for the LM head, whose CTAs with
+// all rows beyond the live row count exit at once.
 constexpr int kBN = 128, kStages = 4;
 constexpr int kSmallRows = 256;  // GEMMs with at most this many rows use the few-rows tiles
 using Big = TcShape<kBN, 2, kStages>;
 using Small = TcShape<kBN, 1, kStages>;
-using SmallGlu = TcShape<64, 1, kStages>;
 
 }  // namespace
 
@@ -42,9 +45,10 @@ struct TcPlan {
     const void *h, *o, *act;
     CUtensorMap map_h, map_o, map_act;        // 256-row boxes
     CUtensorMap map_h1, map_o1, map_act1;     // 128-row boxes
+    CUtensorMap map_h32, map_o32, map_act32;  // 32-row boxes: token operand of the swapped kernel
     std::unordered_map<const void*, CUtensorMap> wmap;   // weight pointer -> map (box rows = tile N or N/2)
-    std::unordered_map<const void*, CUtensorMap> wmap1;  // gate / up maps for the 64-wide SwiGLU tile
     int* err;
+    int sms;
 };
 
 
@@ -68,7 +72,8 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
     bool ok = make_map(&p->map_h, h, rows_full, dm.D, Big::BM) && make_map(&p->map_o, o, rows_full, HD, Big::BM) &&
               make_map(&p->map_act, act, rows_full, dm.F, Big::BM) &&
               make_map(&p->map_h1, h, rows_full, dm.D, Small::BM) && make_map(&p->map_o1, o, rows_full, HD, Small::BM) &&
-              make_map(&p->map_act1, act, rows_full, dm.F, Small::BM);
+              make_map(&p->map_act1, act, rows_full, dm.F, Small::BM) && make_map(&p->map_h32, h, rows_full, dm.D, 32) &&
+              make_map(&p->map_o32, o, rows_full, HD, 32) && make_map(&p->map_act32, act, rows_full, dm.F, 32);
     for (int l = 0; ok && l < w.L; ++l) {
         CUtensorMap m;
         ok = ok && make_map(&m, w.wqkv[l], dm.qkv, dm.D, kBN);
@@ -79,10 +84,6 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
         p->wmap[w.wgate[l]] = m;
         ok = ok && make_map(&m, w.wup[l], dm.F, dm.D, kBN / 2);
         p->wmap[w.wup[l]] = m;
-        ok = ok && make_map(&m, w.wgate[l], dm.F, dm.D, 32);
-        p->wmap1[w.wgate[l]] = m;
-        ok = ok && make_map(&m, w.wup[l], dm.F, dm.D, 32);
-        p->wmap1[w.wup[l]] = m;
         ok = ok && make_map(&m, w.wdown[l], dm.D, dm.F, kBN);
         p->wmap[w.wdown[l]] = m;
     }
@@ -103,10 +104,14 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
          set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_RESID>, Big::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_QKV>, Big::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL>, Small::SMEM) &&
-         set_smem((const void*)tc_gemm_kernel<64, 1, kStages, EPI_SWIGLU>, SmallGlu::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_LMHEAD>, Small::SMEM) &&
-         set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_RESID>, Small::SMEM) &&
-         set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_QKV>, Small::SMEM);
+         set_smem((const void*)tc_gemmt_kernel<EPI_RESID>, kTSmem) &&
+         set_smem((const void*)tc_gemmt_kernel<EPI_QKV>, kTSmem) &&
+         set_smem((const void*)tc_gemmt_kernel<EPI_SWIGLU>, kTSmem);
+    int dev = 0;
+    p->sms = 0;
+    ok = ok && cudaGetDevice(&dev) == cudaSuccess &&
+         cudaDeviceGetAttribute(&p->sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && p->sms > 0;
     if (!ok) {
         delete p;
         return FOCUS_ERR_CUDA;
@@ -117,39 +122,59 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
 
 void tc_plan_destroy(TcPlan* p) { delete p; }
 
-int tc_splits(const TcPlan* p, int wid, int m_bound) {
-    // few-row GEMMs split K so that about 128 CTAs stream each weight matrix; the split partials are
-    // reduced inside the GEMM by the last CTA of each output tile (at most kMaxReduceSplits of them)
-    if (!p || m_bound > kSmallRows) return 1;
-    switch (wid) {
-        case W_QKV: return 4;
-        case W_O: return 8;
-        case W_DOWN: return 8;
-        default: return 1;
+int tc_lm_tiles(const TcPlan* p) { return p ? (p->dm.V + kBN - 1) / kBN : 0; }
+
+namespace {
+
+// Swapped GEMM: 128-feature tiles x 64-token tiles, split K over a cluster of 1, 2, 4 or 8 CTAs so that
+// with one live token tile about one CTA per SM streams the weight matrix (each slice keeps at least one
+// K block).
+int tc_gemm_swapped(TcPlan* p, Epi epi, GemmArgs g, cudaStream_t s) {
+    const CUtensorMap* x = g.A == p->h ? &p->map_h32 : g.A == p->o ? &p->map_o32 : &p->map_act32;
+    const CUtensorMap* w = &p->wmap.find(g.B)->second;  // 128-row boxes; 64-row boxes for gate / up
+    const CUtensorMap* w2 = epi == EPI_SWIGLU ? &p->wmap.find(g.B2)->second : w;
+    const int n_tiles = epi == EPI_SWIGLU ? g.N / 64 : g.N / 128;
+    const int m_tiles = (g.M_bound + kTNT - 1) / kTNT;
+    const int want = (2 * p->sms + n_tiles) / (2 * n_tiles);
+    int splits = 1;
+    while (splits * 2 <= want && splits * 2 <= kTMaxSplits && splits * 2 <= g.K / BK) splits *= 2;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(splits, n_tiles, m_tiles);
+    cfg.blockDim = dim3(192, 1, 1);
+    cfg.dynamicSmemBytes = kTSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    switch (epi) {
+        case EPI_RESID: e = cudaLaunchKernelEx(&cfg, tc_gemmt_kernel<EPI_RESID>, *w, *w2, *x, g, p->err); break;
+        case EPI_QKV: e = cudaLaunchKernelEx(&cfg, tc_gemmt_kernel<EPI_QKV>, *w, *w2, *x, g, p->err); break;
+        default: e = cudaLaunchKernelEx(&cfg, tc_gemmt_kernel<EPI_SWIGLU>, *w, *w2, *x, g, p->err); break;
     }
+    return e == cudaSuccess ? 1 : -1;
 }
 
-int tc_lm_tiles(const TcPlan* p) { return p ? (p->dm.V + kBN - 1) / kBN : 0; }
+}  // namespace
 
 int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g0, cudaStream_t s) {
     if (g0.M_bound <= 0) return 0;
     GemmArgs g = g0;
     const bool small = g.M_bound <= kSmallRows;
+    if (small && (epi == EPI_RESID || epi == EPI_QKV || epi == EPI_SWIGLU)) return tc_gemm_swapped(p, epi, g, s);
     const CUtensorMap* a = g.A == p->h ? (small ? &p->map_h1 : &p->map_h)
                          : g.A == p->o ? (small ? &p->map_o1 : &p->map_o)
                                        : (small ? &p->map_act1 : &p->map_act);
     const CUtensorMap* b = &p->wmap.find(g.B)->second;
-    const CUtensorMap* b2 = b;
-    if (epi == EPI_SWIGLU) {
-        auto& wm = small ? p->wmap1 : p->wmap;
-        b = &wm.find(g.B)->second;
-        b2 = &wm.find(g.B2)->second;
-    }
+    const CUtensorMap* b2 = epi == EPI_SWIGLU ? &p->wmap.find(g.B2)->second : b;
     int splits = (epi == EPI_PARTIAL || epi == EPI_RESID || epi == EPI_QKV) ? g.splits : 1;
     if (splits > g.K / BK) splits = g.K / BK;  // every split slice gets at least one K block
     if (splits < 1) splits = 1;
-    const int glu_cols = small ? 32 : kBN / 2;  // output columns per SwiGLU tile
-    const int n_tiles = epi == EPI_SWIGLU ? g.N / glu_cols : (g.N + kBN - 1) / kBN;
+    const int n_tiles = epi == EPI_SWIGLU ? g.N / (kBN / 2) : (g.N + kBN - 1) / kBN;
     if (epi == EPI_LMHEAD) {
         g.n_tiles = n_tiles;
         g.tile_n = kBN;
@@ -157,24 +182,10 @@ int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g0, cudaStream_t s) {
     const int bm = small ? Small::BM : Big::BM;
     dim3 grid(n_tiles, (g.M_bound + bm - 1) / bm, splits);
     (void)wid;
-    if (small) {
-        switch (epi) {
-            case EPI_PARTIAL:
-                tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
-                break;
-            case EPI_SWIGLU:
-                tc_gemm_kernel<64, 1, kStages, EPI_SWIGLU><<<grid, 192, SmallGlu::SMEM, s>>>(*a, *b, *b2, g, p->err);
-                break;
-            case EPI_LMHEAD:
-                tc_gemm_kernel<kBN, 1, kStages, EPI_LMHEAD><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
-                break;
-            case EPI_RESID:
-                tc_gemm_kernel<kBN, 1, kStages, EPI_RESID><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
-                break;
-            case EPI_QKV:
-                tc_gemm_kernel<kBN, 1, kStages, EPI_QKV><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
-                break;
-        }
+    if (small && epi == EPI_LMHEAD) {
+        tc_gemm_kernel<kBN, 1, kStages, EPI_LMHEAD><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
+    } else if (small && epi == EPI_PARTIAL) {
+        tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
     } else {
         switch (epi) {
             case EPI_PARTIAL:

@@ -23,7 +23,6 @@ struct TcPlan;
 int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, void* o, void* act, int rows_full,
                    int rows_c, int lm_tiles_cap, int* err);
 void tc_plan_destroy(TcPlan* p);
-int tc_splits(const TcPlan* p, int wid, int m_bound);
 int tc_lm_tiles(const TcPlan* p);
 int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g, cudaStream_t s);
 
