@@ -38,6 +38,7 @@ __device__ __forceinline__ const T* key_row(const AttnArgs& a, int b, int g, int
 
 template <typename T>
 __global__ void __launch_bounds__(kAttnWarps * 32) attention_simt_kernel(AttnArgs a) {
+    pdl_entry();
     extern __shared__ float smem[];
     const int b = blockIdx.x, g = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -138,8 +139,7 @@ int launch_attention(const AttnArgs& a, cudaStream_t s) {
     if (smem > 48 * 1024)
         cudaFuncSetAttribute(attention_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 grid(a.N, a.Hkv);
-    attention_simt_kernel<T><<<grid, kAttnWarps * 32, smem, s>>>(a);
-    return 1;
+    return launched(launch_pdl(attention_simt_kernel<T>, grid, dim3(kAttnWarps * 32), smem, s, 0, a));
 }
 
 template int launch_attention<float>(const AttnArgs&, cudaStream_t);

@@ -133,6 +133,7 @@ template <bool FULL>
 __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_constant__ CUtensorMap pool_map,
                                                               const __grid_constant__ CUtensorMap ibc_map, AttnArgs a,
                                                               int q_tiles) {
+    pdl_entry();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* kv = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(8) uint64_t full_bar[kStages];
@@ -581,10 +582,8 @@ int launch_attention_tc(const AttnArgs& a, int q_tiles, cudaStream_t s) {
     }
     dim3 grid(a.N, a.Hkv * a.pieces, q_tiles);
     if (a.row_offsets == nullptr)
-        attention_tc_kernel<true><<<grid, 128, smem, s>>>(pool_map, ibc_map, a, q_tiles);
-    else
-        attention_tc_kernel<false><<<grid, 128, smem, s>>>(pool_map, ibc_map, a, q_tiles);
-    return 1;
+        return launched(launch_pdl(attention_tc_kernel<true>, grid, dim3(128), smem, s, 0, pool_map, ibc_map, a, q_tiles));
+    return launched(launch_pdl(attention_tc_kernel<false>, grid, dim3(128), smem, s, 0, pool_map, ibc_map, a, q_tiles));
 }
 
 }  // namespace focus

@@ -20,6 +20,15 @@ template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __flo
 
 __device__ __forceinline__ void raise_err(int* err, int bit) { atomicOr(err, bit); }
 
+// Programmatic dependent launch: every kernel of the step is launched so that it may start while its
+// predecessor drains.  On entry it lets its own successor launch, then waits until the predecessor has
+// completed and its memory is visible; nothing is read or written before that wait.  (Without a
+// programmatic launch both are no-ops.)
+__device__ __forceinline__ void pdl_entry() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(kCombineThreads) lm_combine_kernel(const float
                                                                      const int32_t* __restrict__ n_rows,
                                                                      float* __restrict__ row_conf,
                                                                      int32_t* __restrict__ row_top) {
+    pdl_entry();
     __shared__ float wm[kCombineThreads / 32], ws[kCombineThreads / 32];
     __shared__ int wa[kCombineThreads / 32];
     const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -83,6 +84,7 @@ __global__ void __launch_bounds__(kCombineThreads) lm_combine_kernel(const float
 }
 
 __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(DecodeArgs a) {
+    pdl_entry();
     __shared__ float conf_s[64];
     __shared__ int top_s[64];
     const int b = blockIdx.x;
@@ -149,15 +151,13 @@ bool configure_select_decode_kernels() {
 
 int launch_lm_combine(const DecodeArgs& a, int rows_bound, const int32_t* n_rows, cudaStream_t s) {
     if (rows_bound <= 0) return 0;
-    lm_combine_kernel<<<rows_bound, kCombineThreads, 0, s>>>(a.lm_max, a.lm_sum, a.lm_arg, a.n_tiles, n_rows,
-                                                            a.row_conf, a.row_top);
-    return 1;
+    return launched(launch_pdl(lm_combine_kernel, dim3(rows_bound), dim3(kCombineThreads), 0, s, 0, a.lm_max, a.lm_sum,
+                               a.lm_arg, a.n_tiles, n_rows, a.row_conf, a.row_top));
 }
 
 int launch_decode(const DecodeArgs& a, cudaStream_t s) {
     if (a.N <= 0) return 0;
-    decode_kernel<<<a.N, kDecodeWarps * 32, 0, s>>>(a);
-    return 1;
+    return launched(launch_pdl(decode_kernel, dim3(a.N), dim3(kDecodeWarps * 32), 0, s, 0, a));
 }
 
 }  // namespace focus

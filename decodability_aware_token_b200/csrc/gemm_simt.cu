@@ -16,6 +16,7 @@ constexpr int TM = 64, TN = 64, TK = 16;
 
 template <typename T, int EPI>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs g) {
+    pdl_entry();
     __shared__ float As[TK][TM + 4];
     __shared__ float Bs[TK][TN + 4];
     __shared__ float Bs2[EPI == EPI_SWIGLU ? TK : 1][TN + 4];
@@ -138,11 +139,11 @@ int launch_gemm_simt(Epi epi, const GemmArgs& g, cudaStream_t s) {
     GemmArgs a = g;
     if (epi != EPI_PARTIAL) a.splits = 1;
     switch (epi) {
-        case EPI_PARTIAL: gemm_simt_kernel<T, EPI_PARTIAL><<<grid, 256, 0, s>>>(a); break;
-        case EPI_SWIGLU: gemm_simt_kernel<T, EPI_SWIGLU><<<grid, 256, 0, s>>>(a); break;
-        case EPI_LMHEAD: gemm_simt_kernel<T, EPI_LMHEAD><<<grid, 256, 0, s>>>(a); break;
+        case EPI_PARTIAL: return launched(launch_pdl(gemm_simt_kernel<T, EPI_PARTIAL>, grid, dim3(256), 0, s, 0, a));
+        case EPI_SWIGLU: return launched(launch_pdl(gemm_simt_kernel<T, EPI_SWIGLU>, grid, dim3(256), 0, s, 0, a));
+        case EPI_LMHEAD: return launched(launch_pdl(gemm_simt_kernel<T, EPI_LMHEAD>, grid, dim3(256), 0, s, 0, a));
+        default: return -1;
     }
-    return 1;
 }
 
 template int launch_gemm_simt<float>(Epi, const GemmArgs&, cudaStream_t);

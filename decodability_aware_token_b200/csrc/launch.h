@@ -22,6 +22,34 @@ bool configure_select_decode_kernels();
 bool configure_select_kernel();
 bool configure_simt_gemm_kernels();
 
+// Launch with programmatic stream serialisation (the kernel starts with pdl_entry()); cluster_x > 0
+// launches clusters of cluster_x CTAs along x.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              unsigned cluster_x, Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+inline int launched(cudaError_t e) { return e == cudaSuccess ? 1 : -1; }
+
 struct Dims {
     int L, D, Hq, Hkv, d, F, V, qkv;  // qkv = (Hq + 2 Hkv) d
     float eps;

@@ -18,6 +18,7 @@ __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(const int32_t*
                                                                   const T* __restrict__ embed,
                                                                   const T* __restrict__ gamma, float eps, int D,
                                                                   float* __restrict__ x, T* __restrict__ h, int* err) {
+    pdl_entry();
     __shared__ float red[32];
     const int r = blockIdx.x, tid = threadIdx.x;
     int tok = tokens[r];
@@ -48,6 +49,7 @@ __global__ void __launch_bounds__(kNormThreads) residual_norm_kernel(
     const float* __restrict__ x_in, const int32_t* __restrict__ src_map, const int32_t* __restrict__ n_rows_dev,
     const float* __restrict__ part, int n_splits, size_t part_stride, float* x_out, const T* __restrict__ gamma,
     float eps, int D, T* __restrict__ h_out) {
+    pdl_entry();
     __shared__ float red[32];
     const int r = blockIdx.x, tid = threadIdx.x;
     if (n_rows_dev && r >= *n_rows_dev) return;
@@ -98,6 +100,7 @@ __global__ void __launch_bounds__(kRowThreads) qkv_finalize_kernel(const float* 
                                                                    int max_prefix, const double* __restrict__ inv_freq,
                                                                    Dims dm, int layer, T* __restrict__ q_out,
                                                                    T* __restrict__ ibc, int* err) {
+    pdl_entry();
     extern __shared__ float cs[];  // [d/2] cos, [d/2] sin
     const int r = blockIdx.x;
     if (r >= rm.rows()) return;
@@ -157,8 +160,8 @@ template <typename T>
 int launch_embed_norm(const int32_t* tokens, int rows, int V, const T* embed, const T* gamma, float eps, int D,
                        float* x, T* h, int* err, cudaStream_t s) {
     if (rows <= 0) return 0;
-    embed_norm_kernel<T><<<rows, kNormThreads, 0, s>>>(tokens, V, embed, gamma, eps, D, x, h, err);
-    return 1;
+    return launched(launch_pdl(embed_norm_kernel<T>, dim3(rows), dim3(kNormThreads), 0, s, 0, tokens, V, embed, gamma,
+                               eps, D, x, h, err));
 }
 
 template <typename T>
@@ -166,9 +169,8 @@ int launch_residual_norm(const float* x_in, const int32_t* src_map, const int32_
                           const float* part, int n_splits, size_t part_stride, float* x_out, const T* gamma,
                           float eps, int D, T* h_out, cudaStream_t s) {
     if (rows_bound <= 0) return 0;
-    residual_norm_kernel<T><<<rows_bound, kNormThreads, 0, s>>>(x_in, src_map, n_rows_dev, part, n_splits, part_stride,
-                                                                x_out, gamma, eps, D, h_out);
-    return 1;
+    return launched(launch_pdl(residual_norm_kernel<T>, dim3(rows_bound), dim3(kNormThreads), 0, s, 0, x_in, src_map,
+                               n_rows_dev, part, n_splits, part_stride, x_out, gamma, eps, D, h_out));
 }
 
 template <typename T>
@@ -176,9 +178,9 @@ int launch_qkv_finalize(const float* part, int n_splits, size_t part_stride, Row
                          int max_prefix, const double* inv_freq, Dims dm, int layer, T* q_out, T* ibc, int* err,
                          cudaStream_t s) {
     if (rm.rows_static <= 0) return 0;
-    qkv_finalize_kernel<T><<<rm.rows_static, kRowThreads, dm.d * sizeof(float), s>>>(
-        part, n_splits, part_stride, rm, prefix_len, max_prefix, inv_freq, dm, layer, q_out, ibc, err);
-    return 1;
+    return launched(launch_pdl(qkv_finalize_kernel<T>, dim3(rm.rows_static), dim3(kRowThreads), dm.d * sizeof(float), s,
+                               0, part, n_splits, part_stride, rm, prefix_len, max_prefix, inv_freq, dm, layer, q_out,
+                               ibc, err));
 }
 
 bool configure_rows_kernels() {

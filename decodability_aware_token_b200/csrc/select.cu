@@ -26,6 +26,7 @@ __device__ __forceinline__ bool key_less(bool forced, bool ma, float da, int ja,
 }
 
 __global__ void __launch_bounds__(1024) select_kernel(SelectArgs a) {
+    pdl_entry();
     extern __shared__ int32_t sh[];  // [N] kept counts, [N + 1] offsets
     int32_t* kc_s = sh;
     int32_t* off_s = sh + a.N;
@@ -148,8 +149,7 @@ int launch_select(const SelectArgs& a, cudaStream_t s) {
     if (a.N <= 0) return 0;
     const size_t smem = sizeof(int32_t) * (2 * (size_t)a.N + 1);
     if (smem > 48 * 1024) cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    select_kernel<<<1, 1024, smem, s>>>(a);
-    return 1;
+    return launched(launch_pdl(select_kernel, dim3(1), dim3(1024), smem, s, 0, a));
 }
 
 }  // namespace focus

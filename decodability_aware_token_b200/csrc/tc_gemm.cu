@@ -49,6 +49,7 @@ struct TcPlan {
     std::unordered_map<const void*, CUtensorMap> wmap;   // weight pointer -> map (box rows = tile N or N/2)
     int* err;
     int sms;
+    int max_clusters[kTMaxSplits + 1];  // co-resident clusters of the swapped kernel with s CTAs (0: not launchable)
 };
 
 
@@ -104,14 +105,37 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
          set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_RESID>, Big::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_QKV>, Big::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL>, Small::SMEM) &&
-         set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_LMHEAD>, Small::SMEM) &&
          set_smem((const void*)tc_gemmt_kernel<EPI_RESID>, kTSmem) &&
          set_smem((const void*)tc_gemmt_kernel<EPI_QKV>, kTSmem) &&
-         set_smem((const void*)tc_gemmt_kernel<EPI_SWIGLU>, kTSmem);
+         set_smem((const void*)tc_gemmt_kernel<EPI_SWIGLU>, kTSmem) &&
+         set_smem((const void*)tc_gemmt_kernel<EPI_LMHEAD>, kTSmem);
     int dev = 0;
     p->sms = 0;
     ok = ok && cudaGetDevice(&dev) == cudaSuccess &&
          cudaDeviceGetAttribute(&p->sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && p->sms > 0;
+    // how many clusters of each size fit at once (a cluster's CTAs share one GPC, so this is not
+    // simply SMs / size)
+    p->max_clusters[0] = 0;
+    for (int cs = 1; ok && cs <= kTMaxSplits; ++cs) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(cs, 1, 1);
+        cfg.blockDim = dim3(192, 1, 1);
+        cfg.dynamicSmemBytes = kTSmem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, tc_gemmt_kernel<EPI_RESID>, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();  // a cluster shape the device does not take is simply not used
+            n = 0;
+        }
+        p->max_clusters[cs] = n;
+    }
+    ok = ok && p->max_clusters[1] > 0;
     if (!ok) {
         delete p;
         return FOCUS_ERR_CUDA;
@@ -126,35 +150,41 @@ int tc_lm_tiles(const TcPlan* p) { return p ? (p->dm.V + kBN - 1) / kBN : 0; }
 
 namespace {
 
-// Swapped GEMM: 128-feature tiles x 64-token tiles, split K over a cluster of 1, 2, 4 or 8 CTAs so that
-// with one live token tile about one CTA per SM streams the weight matrix (each slice keeps at least one
-// K block).
+// Swapped GEMM: 128-feature tiles x all live tokens, split K over a cluster of 1..8 CTAs (each slice keeps
+// at least one K block).  The LM head (many feature tiles) does not split.
 int tc_gemm_swapped(TcPlan* p, Epi epi, GemmArgs g, cudaStream_t s) {
     const CUtensorMap* x = g.A == p->h ? &p->map_h32 : g.A == p->o ? &p->map_o32 : &p->map_act32;
     const CUtensorMap* w = &p->wmap.find(g.B)->second;  // 128-row boxes; 64-row boxes for gate / up
     const CUtensorMap* w2 = epi == EPI_SWIGLU ? &p->wmap.find(g.B2)->second : w;
-    const int n_tiles = epi == EPI_SWIGLU ? g.N / 64 : g.N / 128;
-    const int m_tiles = (g.M_bound + kTNT - 1) / kTNT;
-    const int want = (2 * p->sms + n_tiles) / (2 * n_tiles);
+    const int n_tiles = epi == EPI_SWIGLU ? g.N / 64 : (g.N + 127) / 128;
+    // split K so that the busiest SM streams the least: with every cluster resident at once (one wave),
+    // the busiest SM holds ceil(n_tiles * s / SMs) CTAs of nk / s K blocks each; ties go to fewer slices
     int splits = 1;
-    while (splits * 2 <= want && splits * 2 <= kTMaxSplits && splits * 2 <= g.K / BK) splits *= 2;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(splits, n_tiles, m_tiles);
-    cfg.blockDim = dim3(192, 1, 1);
-    cfg.dynamicSmemBytes = kTSmem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    if (epi != EPI_LMHEAD) {
+        double best = 0.0;
+        for (int cs = 1; cs <= kTMaxSplits && cs <= g.K / BK; ++cs) {
+            if (n_tiles > p->max_clusters[cs]) continue;
+            const double load = (double)((n_tiles * cs + p->sms - 1) / p->sms) / cs;
+            if (cs == 1 || load < best - 1e-9) {
+                best = load;
+                splits = cs;
+            }
+        }
+    }
+    if (epi == EPI_LMHEAD) {
+        g.n_tiles = n_tiles;
+        g.tile_n = 128;
+    }
+    const dim3 grid(splits, n_tiles, 1), blk(192);
+    const unsigned cx = (unsigned)splits;
     cudaError_t e;
     switch (epi) {
-        case EPI_RESID: e = cudaLaunchKernelEx(&cfg, tc_gemmt_kernel<EPI_RESID>, *w, *w2, *x, g, p->err); break;
-        case EPI_QKV: e = cudaLaunchKernelEx(&cfg, tc_gemmt_kernel<EPI_QKV>, *w, *w2, *x, g, p->err); break;
-        default: e = cudaLaunchKernelEx(&cfg, tc_gemmt_kernel<EPI_SWIGLU>, *w, *w2, *x, g, p->err); break;
+        case EPI_RESID: e = launch_pdl(tc_gemmt_kernel<EPI_RESID>, grid, blk, kTSmem, s, cx, *w, *w2, *x, g, p->err); break;
+        case EPI_QKV: e = launch_pdl(tc_gemmt_kernel<EPI_QKV>, grid, blk, kTSmem, s, cx, *w, *w2, *x, g, p->err); break;
+        case EPI_LMHEAD:
+            e = launch_pdl(tc_gemmt_kernel<EPI_LMHEAD>, grid, blk, kTSmem, s, cx, *w, *w2, *x, g, p->err);
+            break;
+        default: e = launch_pdl(tc_gemmt_kernel<EPI_SWIGLU>, grid, blk, kTSmem, s, cx, *w, *w2, *x, g, p->err); break;
     }
     return e == cudaSuccess ? 1 : -1;
 }
@@ -165,7 +195,7 @@ int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g0, cudaStream_t s) {
     if (g0.M_bound <= 0) return 0;
     GemmArgs g = g0;
     const bool small = g.M_bound <= kSmallRows;
-    if (small && (epi == EPI_RESID || epi == EPI_QKV || epi == EPI_SWIGLU)) return tc_gemm_swapped(p, epi, g, s);
+    if (small && epi != EPI_PARTIAL) return tc_gemm_swapped(p, epi, g, s);
     const CUtensorMap* a = g.A == p->h ? (small ? &p->map_h1 : &p->map_h)
                          : g.A == p->o ? (small ? &p->map_o1 : &p->map_o)
                                        : (small ? &p->map_act1 : &p->map_act);
@@ -182,30 +212,28 @@ int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g0, cudaStream_t s) {
     const int bm = small ? Small::BM : Big::BM;
     dim3 grid(n_tiles, (g.M_bound + bm - 1) / bm, splits);
     (void)wid;
-    if (small && epi == EPI_LMHEAD) {
-        tc_gemm_kernel<kBN, 1, kStages, EPI_LMHEAD><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
-    } else if (small && epi == EPI_PARTIAL) {
-        tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL><<<grid, 192, Small::SMEM, s>>>(*a, *b, *b2, g, p->err);
-    } else {
-        switch (epi) {
-            case EPI_PARTIAL:
-                tc_gemm_kernel<kBN, 2, kStages, EPI_PARTIAL><<<grid, 192, Big::SMEM, s>>>(*a, *b, *b2, g, p->err);
-                break;
-            case EPI_SWIGLU:
-                tc_gemm_kernel<kBN, 2, kStages, EPI_SWIGLU><<<grid, 192, Big::SMEM, s>>>(*a, *b, *b2, g, p->err);
-                break;
-            case EPI_LMHEAD:
-                tc_gemm_kernel<kBN, 2, kStages, EPI_LMHEAD><<<grid, 192, Big::SMEM, s>>>(*a, *b, *b2, g, p->err);
-                break;
-            case EPI_RESID:
-                tc_gemm_kernel<kBN, 2, kStages, EPI_RESID><<<grid, 192, Big::SMEM, s>>>(*a, *b, *b2, g, p->err);
-                break;
-            case EPI_QKV:
-                tc_gemm_kernel<kBN, 2, kStages, EPI_QKV><<<grid, 192, Big::SMEM, s>>>(*a, *b, *b2, g, p->err);
-                break;
-        }
+    const dim3 blk(192);
+    if (small)  // EPI_PARTIAL
+        return launched(launch_pdl(tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL>, grid, blk, Small::SMEM, s, 0, *a, *b, *b2,
+                                   g, p->err));
+    switch (epi) {
+        case EPI_PARTIAL:
+            return launched(launch_pdl(tc_gemm_kernel<kBN, 2, kStages, EPI_PARTIAL>, grid, blk, Big::SMEM, s, 0, *a, *b,
+                                       *b2, g, p->err));
+        case EPI_SWIGLU:
+            return launched(launch_pdl(tc_gemm_kernel<kBN, 2, kStages, EPI_SWIGLU>, grid, blk, Big::SMEM, s, 0, *a, *b,
+                                       *b2, g, p->err));
+        case EPI_LMHEAD:
+            return launched(launch_pdl(tc_gemm_kernel<kBN, 2, kStages, EPI_LMHEAD>, grid, blk, Big::SMEM, s, 0, *a, *b,
+                                       *b2, g, p->err));
+        case EPI_RESID:
+            return launched(launch_pdl(tc_gemm_kernel<kBN, 2, kStages, EPI_RESID>, grid, blk, Big::SMEM, s, 0, *a, *b,
+                                       *b2, g, p->err));
+        case EPI_QKV:
+            return launched(launch_pdl(tc_gemm_kernel<kBN, 2, kStages, EPI_QKV>, grid, blk, Big::SMEM, s, 0, *a, *b, *b2,
+                                       g, p->err));
     }
-    return 1;
+    return -1;
 }
 
 }  // namespace focus

@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
                                                          const __grid_constant__ CUtensorMap tmB,
                                                          const __grid_constant__ CUtensorMap tmB2, GemmArgs g,
                                                          int* err) {
+    pdl_entry();
     using S = TcShape<BN, MSUB, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -496,30 +497,34 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
 }
 
 // ------------------------------------------------------------------ swapped GEMM for few rows
-// For the kept rows (a few dozen tokens) the GEMMs stream weights.  The product is computed transposed,
-// D^T = W X^T: the 128 output features of a tile sit on the MMA's M side and up to 64 tokens on its
-// N side, so no tensor work or operand bytes go to absent rows.  A stage holds the 16 KB weight tile
-// and only the live 32-token boxes of the activations (token rows of the 8 KB tile that were not loaded
-// only reach accumulator columns that are never read).
+// For the kept rows (at most 256 tokens, typically a few dozen) the GEMMs stream weights.  The product is
+// computed transposed, D^T = W X^T: the 128 output features of a tile sit on the MMA's M side and every
+// live token on its N side (N = the live count rounded up to 32, at most 256), so one CTA covers all
+// tokens of its feature tile, no CTA is spent on absent rows and no tensor work or operand bytes go to
+// them.  A stage holds the 16 KB weight tile and one 4 KB box per live 32-token group; the 100 KB
+// operand ring (two CTAs per SM) holds 5 stages for up to 32 tokens.
 //
 // Split K runs inside a thread-block cluster: the `splits` CTAs of one output tile are the cluster's
-// ranks, each accumulates its K slice in TMEM and parks it in its own shared memory as [token][feature]
-// fp32; after a cluster barrier rank r sums the slices of its share of the tokens in rank order through
+// ranks, each accumulates its K slice in TMEM and parks it (128 tokens at a time) in its own shared memory
+// as [token][feature] fp32; after a cluster barrier rank r sums the slices of its share of the tokens in rank order through
 // distributed shared memory and applies the epilogue to them.  No partial sums go through global memory
 // and no CTA waits on an arrival counter.  Epilogue threads own one output feature each, so for every
 // token a warp touches 32 consecutive features.  Pairs of features f and f + 64 (the RoPE halves of a
-// head; gate and up of SwiGLU, loaded as two 64-row weight boxes) are both in the parked tile.
+// head; gate and up of SwiGLU, loaded as two 64-row weight boxes) are both in the parked tile.  The
+// LM-head epilogue (no split) reduces each token's 128 vocabulary features of the tile to the max
+// logit, sum exp(z - max) and first argmax, so no logits reach global memory.
 //
-// Grid: (splits, feature tiles, token tiles), cluster (splits, 1, 1); the token tiles beyond the live
-// row count exit as whole clusters before any barrier.
-constexpr int kTNT = 64;                         // tokens per CTA (MMA N)
-constexpr int kTStages = 4;
+// Grid: (splits, feature tiles), cluster (splits, 1, 1).
+constexpr int kTMaxTok = 256;                    // tokens per CTA (MMA N <= 256)
 constexpr int kTW = 128 * BK * 2;                // weight tile bytes (16 KB)
-constexpr int kTX = kTNT * BK * 2;               // token tile bytes (8 KB)
-constexpr int kTStage = kTW + kTX;
-constexpr int kTSmem = kTStages * kTStage + 1024;
+constexpr int kTXBox = 32 * BK * 2;              // one 32-token box of the token tile (4 KB)
+constexpr int kTRing = 100 * 1024;               // operand ring bytes (two CTAs per SM)
+constexpr int kTMaxStages = kTRing / (kTW + kTXBox);
+constexpr int kTSmem = kTRing + 1024;            // + alignment slack
 constexpr int kTMaxSplits = 8;                   // portable cluster size
-static_assert(kTNT * 128 * 4 <= kTStages * kTStage, "parked tile reuses the operand ring");
+constexpr int kTChunk = 128;                     // tokens parked at a time
+constexpr int kTPark = 129;                      // parked tile row stride (odd: token-major scans are conflict free)
+static_assert(kTChunk * kTPark * 4 <= kTRing, "parked tile reuses the operand ring");
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -545,17 +550,20 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap tmW2,
                                                           const __grid_constant__ CUtensorMap tmX, GemmArgs g,
                                                           int* err) {
+    pdl_entry();
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full_bar[kTStages];
-    __shared__ __align__(8) uint64_t empty_bar[kTStages];
+    __shared__ __align__(8) uint64_t full_bar[kTMaxStages];
+    __shared__ __align__(8) uint64_t empty_bar[kTMaxStages];
     __shared__ __align__(8) uint64_t accum_bar;
     __shared__ uint32_t tmem_slot;
 
-    const int M = g.M_dev ? *g.M_dev : g.M_bound;
-    const int m0 = blockIdx.z * kTNT;
-    if (m0 >= M) return;  // the whole cluster (same token tile), before any barrier or TMEM use
-    const int m_live = min(kTNT, M - m0);
-    const int x_boxes = (m_live + 31) / 32;
+    const int M = min(g.M_dev ? *g.M_dev : g.M_bound, kTMaxTok);  // the launcher keeps M_bound <= 256
+    if (M <= 0) return;  // the whole grid, before any barrier or TMEM use
+    const int x_boxes = (M + 31) / 32;
+    const int n_cols = x_boxes * 32;               // MMA N and TMEM columns read back
+    const uint32_t tmem_cols = n_cols <= 32 ? 32u : n_cols <= 64 ? 64u : n_cols <= 128 ? 128u : 256u;
+    const int stage_bytes = kTW + x_boxes * kTXBox;  // a multiple of 1024 (swizzle atom alignment)
+    const int nst = min(kTMaxStages, kTRing / stage_bytes);
     const int n_tile = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -564,11 +572,11 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
     const int nk_all = g.K / BK;
     const int kb0 = (int)((long long)nk_all * split / splits);
     const int nk = (int)((long long)nk_all * (split + 1) / splits) - kb0;
-    // output features of the tile: 128 (QKV: one head; residual GEMMs), or 64 gate + 64 up (SwiGLU)
+    // output features of the tile: 128 (QKV: one head; residual GEMMs; LM head), or 64 gate + 64 up (SwiGLU)
     const int fbase = EPI == EPI_SWIGLU ? n_tile * 64 : n_tile * 128;
 
     if (threadIdx.x == 0) {
-        for (int st = 0; st < kTStages; ++st) {
+        for (int st = 0; st < nst; ++st) {
             mbar_init(&full_bar[st], 1);
             mbar_init(&empty_bar[st], 1);
         }
@@ -577,7 +585,7 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
-                     "r"((uint32_t)kTNT)
+                     "r"(tmem_cols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -585,7 +593,7 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
-    float* park = reinterpret_cast<float*>(smem);  // [kTNT tokens][128 features], once the ring is idle
+    float* park = reinterpret_cast<float*>(smem);  // [token][kTPark] features, once the ring is idle
 
     if (warp == 0) {
         if (lane == 0) {
@@ -593,37 +601,37 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
             asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(&tmX) : "memory");
             if (EPI == EPI_SWIGLU) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW2) : "memory");
-            const uint32_t bytes = (uint32_t)(kTW + x_boxes * 32 * BK * 2);
+            const uint32_t bytes = (uint32_t)stage_bytes;
             int issued = 0;
             for (int i = 0; i < nk; ++i) {
-                const int st = i % kTStages;
-                const uint32_t ph = (uint32_t)(i / kTStages) & 1u;
+                const int st = i % nst;
+                const uint32_t ph = (uint32_t)(i / nst) & 1u;
                 if (!mbar_wait(&empty_bar[st], ph ^ 1u, err)) break;
-                uint8_t* w_dst = smem + st * kTStage;
+                uint8_t* w_dst = smem + st * stage_bytes;
                 uint8_t* x_dst = w_dst + kTW;
                 mbar_expect_tx(&full_bar[st], bytes);
                 const int kx = (kb0 + i) * BK;
                 tma_load_2d(&tmW, &full_bar[st], w_dst, kx, fbase);
                 if (EPI == EPI_SWIGLU) tma_load_2d(&tmW2, &full_bar[st], w_dst + kTW / 2, kx, fbase);
                 for (int bx = 0; bx < x_boxes; ++bx)
-                    tma_load_2d(&tmX, &full_bar[st], x_dst + bx * 32 * BK * 2, kx, m0 + bx * 32);
+                    tma_load_2d(&tmX, &full_bar[st], x_dst + bx * kTXBox, kx, bx * 32);
                 ++issued;
             }
             // never leave with copies in flight: wait (bounded) for the last stages issued
-            for (int i = issued - 1; i >= 0 && i >= issued - kTStages; --i)
-                mbar_wait(&full_bar[i % kTStages], (uint32_t)(i / kTStages) & 1u, err);
+            for (int i = issued - 1; i >= 0 && i >= issued - nst; --i)
+                mbar_wait(&full_bar[i % nst], (uint32_t)(i / nst) & 1u, err);
         }
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
-            // ---- MMA issuer (one thread): 128 features x 64 tokens per instruction
-            constexpr uint32_t idesc = idesc_bf16(128, kTNT);
+            // ---- MMA issuer (one thread): 128 features x n_cols tokens per instruction
+            const uint32_t idesc = idesc_bf16(128, n_cols);
             for (int i = 0; i < nk; ++i) {
-                const int st = i % kTStages;
-                const uint32_t ph = (uint32_t)(i / kTStages) & 1u;
+                const int st = i % nst;
+                const uint32_t ph = (uint32_t)(i / nst) & 1u;
                 if (!mbar_wait(&full_bar[st], ph, err)) break;
                 tc_fence_after();
-                const uint32_t w_addr = smem_u32(smem + st * kTStage);
+                const uint32_t w_addr = smem_u32(smem + st * stage_bytes);
                 const uint32_t x_addr = w_addr + kTW;
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
@@ -634,37 +642,63 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
             mma_commit(&accum_bar);
         }
         __syncwarp();
-    } else {
-        // ---- park the accumulators: warp w holds TMEM lanes 32 (w % 4) .. +31, i.e. features f
-        const int f = (warp & 3) * 32 + lane;
-        const bool ok = mbar_wait(&accum_bar, 0, err);
+    }
+    // ---- epilogue warps: accumulators ready?
+    const int f_own = (warp & 3) * 32 + lane;  // warp w holds TMEM lanes 32 (w % 4) .. +31, i.e. features f
+    const uint32_t tbase = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    bool live = false;  // otherwise this slice contributes zeros (a timeout is flagged)
+    if (warp >= 2) {
+        live = mbar_wait(&accum_bar, 0, err) && nk > 0;
         tc_fence_after();
-        const uint32_t tbase = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        const bool live = ok && nk > 0;  // otherwise this slice contributes zeros (a timeout is flagged)
+    }
+    // tokens in chunks of kTChunk, each parked, reduced across the cluster and finished
 #pragma unroll 1
-        for (int c0 = 0; c0 < kTNT; c0 += 32) {
-            if (c0 < m_live) {  // CTA-uniform: all lanes of the warp execute the load
+    for (int c = 0; c < M; c += kTChunk) {
+        const int cm = min(kTChunk, M - c);
+        if (c > 0) cluster_sync_all();  // the previous chunk's parked tiles are no longer read
+        if (warp >= 2) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < cm; c0 += 32) {  // CTA-uniform: all lanes of the warp execute the load
                 float v[32];
-                tmem_ld32(tbase + c0, v);
+                tmem_ld32(tbase + c + c0, v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    if (c0 + i < m_live) park[(c0 + i) * 128 + f] = live ? v[i] : 0.f;
+                    if (c0 + i < cm) park[(c0 + i) * kTPark + f_own] = live ? v[i] : 0.f;
             }
         }
-    }
-    cluster_sync_all();  // every slice of the tile is parked
-
-    if (warp >= 2) {
-        // ---- this rank's tokens [t0, t1): sum the slices in rank order, then the epilogue
+        cluster_sync_all();  // every slice of the chunk is parked
+        if (warp < 2) continue;
         const int e = threadIdx.x - 64;
-        const int t0 = m_live * split / splits, t1 = m_live * (split + 1) / splits;
+        if (EPI == EPI_LMHEAD) {
+            // ---- per token: the tile's max logit, first argmax and sum exp(z - max) (no split)
+            const int n_valid = min(128, g.N - fbase);
+            for (int t = e; t < cm; t += 128) {
+                const float* z = park + t * kTPark;
+                float mx = -CUDART_INF_F;
+                int arg = 0x7fffffff;
+                for (int q = 0; q < n_valid; ++q)
+                    if (z[q] > mx) {
+                        mx = z[q];
+                        arg = fbase + q;
+                    }
+                float se = 0.f;
+                for (int q = 0; q < n_valid; ++q) se += expf(z[q] - mx);
+                const size_t idx = (size_t)(c + t) * g.n_tiles + n_tile;
+                g.lm_max[idx] = mx;
+                g.lm_sum[idx] = se;
+                g.lm_arg[idx] = arg;
+            }
+            continue;
+        }
+        // ---- this rank's tokens [t0, t1) of the chunk: sum the slices in rank order, then the epilogue
+        const int t0 = cm * split / splits, t1 = cm * (split + 1) / splits;
         const uint32_t park_local = smem_u32(park);
         uint32_t peer[kTMaxSplits];
 #pragma unroll
         for (int sp = 0; sp < kTMaxSplits; ++sp) peer[sp] = sp < splits ? cluster_map(park_local, sp) : 0u;
         if (EPI == EPI_RESID) {
             const int f = e;
-            float* xc = g.resid + (size_t)m0 * g.N + fbase + f;
+            float* xc = g.resid + (size_t)c * g.N + fbase + f;
             for (int t = t0; t < t1; t += 4) {
                 float pv[4][kTMaxSplits], xv[4];
 #pragma unroll
@@ -672,7 +706,8 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
                     xv[q] = t + q < t1 ? xc[(size_t)(t + q) * g.N] : 0.f;
 #pragma unroll
                     for (int sp = 0; sp < kTMaxSplits; ++sp)
-                        pv[q][sp] = (sp < splits && t + q < t1) ? ld_cluster_f32(peer[sp] + ((t + q) * 128 + f) * 4) : 0.f;
+                        pv[q][sp] = (sp < splits && t + q < t1) ? ld_cluster_f32(peer[sp] + ((t + q) * kTPark + f) * 4)
+                                                                 : 0.f;
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -694,8 +729,8 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
 #pragma unroll
                     for (int sp = 0; sp < kTMaxSplits; ++sp) {
                         const bool in = sp < splits && tt < t1;
-                        lo_p[q][sp] = in ? ld_cluster_f32(peer[sp] + (tt * 128 + fp) * 4) : 0.f;
-                        hi_p[q][sp] = in ? ld_cluster_f32(peer[sp] + (tt * 128 + fp + 64) * 4) : 0.f;
+                        lo_p[q][sp] = in ? ld_cluster_f32(peer[sp] + (tt * kTPark + fp) * 4) : 0.f;
+                        hi_p[q][sp] = in ? ld_cluster_f32(peer[sp] + (tt * kTPark + fp + 64) * 4) : 0.f;
                     }
                 }
 #pragma unroll
@@ -708,13 +743,14 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
                         a += lo_p[q][sp];
                         bb += hi_p[q][sp];
                     }
+                    const int row = c + tt;
                     if (EPI == EPI_SWIGLU) {
-                        bf16* out = reinterpret_cast<bf16*>(g.act) + (size_t)(m0 + tt) * g.N + fbase + fp;
+                        bf16* out = reinterpret_cast<bf16*>(g.act) + (size_t)row * g.N + fbase + fp;
                         *out = __float2bfloat16_rn(a / (1.f + expf(-a)) * bb);
                     } else {  // EPI_QKV: one head per tile; queries and keys rotate (fp, fp + 64)
                         const int head = n_tile;
                         int b, j, pos;
-                        qkv_row(g, m0 + tt, b, j, pos);
+                        qkv_row(g, row, b, j, pos);
                         float lo = a, hi = bb;
                         if (head < g.Hq + g.Hkv) {
                             float cn, sn;
@@ -722,7 +758,7 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
                             lo = a * cn - bb * sn;
                             hi = bb * cn + a * sn;
                         }
-                        bf16* dst = qkv_dst(g, m0 + tt, head, b, j);
+                        bf16* dst = qkv_dst(g, row, head, b, j);
                         dst[fp] = __float2bfloat16_rn(lo);
                         dst[fp + 64] = __float2bfloat16_rn(hi);
                     }
@@ -734,8 +770,7 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
     cluster_sync_all();  // no rank leaves (or reuses its shared memory) while others still read it
     tc_fence_after();
     if (warp == 1) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)kTNT)
-                     : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols) : "memory");
     }
 }
 
