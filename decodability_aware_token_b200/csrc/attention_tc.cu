@@ -560,10 +560,10 @@ int launch_attention_tc(const AttnArgs& a, int q_tiles, cudaStream_t s) {
     // K|V, head) cache block of B rows is a run of consecutive 256-byte rows
     CUtensorMap pool_map, ibc_map;
     const uint64_t ibc_rows = (uint64_t)a.N * a.L * 2 * a.Hkv * a.B;
-    if (!tc::make_map(&ibc_map, a.ibc, ibc_rows, kD, (uint32_t)a.B)) return -1;
+    if (!tc::make_map(&ibc_map, a.ibc, ibc_rows, kD, (uint32_t)a.B, false)) return -1;
     if (a.n_pages > 0) {
         const uint64_t pool_rows = (uint64_t)a.n_pages * a.L * 2 * a.Hkv * a.page_size;
-        if (!tc::make_map(&pool_map, a.kv_pool, pool_rows, kD, (uint32_t)a.page_size)) return -1;
+        if (!tc::make_map(&pool_map, a.kv_pool, pool_rows, kD, (uint32_t)a.page_size, false)) return -1;
     } else {
         pool_map = ibc_map;  // never used: with no pages every prefix key is invalid
     }
