@@ -168,11 +168,14 @@ def algorithmic_work(kclass: str, case: fs.Case, R: int, kept_per_req, plen, spl
 
 
 def source_digest(kclass: str) -> str:
-    files = {"gemm": ["tc_gemm.cu", "gemm_simt.cu"], "attn": ["attention.cu"], "row": ["rows.cu"],
+    """Digest of the sources that build a kernel class (recorded traffic is used only while it matches)."""
+    shared = ["common.cuh", "launch.h"]
+    files = {"gemm": ["tc_gemm.cu", "tc_gemm_kernel.cuh", "gemm_simt.cu"],
+             "attn": ["attention_tc.cu", "attention.cu", "tc_gemm_kernel.cuh"], "row": ["rows.cu"],
              "qkv": ["rows.cu"], "embed": ["rows.cu"], "select": ["select.cu"], "decode": ["decode.cu"]}
     key = kclass.split("_")[0]
     h = hashlib.sha256()
-    for f in files.get(key, []):
+    for f in files.get(key, []) + shared:
         p = os.path.join(ROOT, "decodability_aware_token_b200", "csrc", f)
         if os.path.exists(p):
             h.update(open(p, "rb").read())
@@ -180,16 +183,19 @@ def source_digest(kclass: str) -> str:
 
 
 def recorded_traffic(kclass: str):
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch of a kernel class from an ncu capture, as recorded in profiles/traffic.md
+    (a table row `| class | source digest | bytes per launch | ... |`); None if absent or stale."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(p):
         return None
-    try:
-        ent = json.load(open(p)).get(kclass)
-    except Exception:
-        return None
-    if not ent or ent.get("source_digest") != source_digest(kclass):
-        return None
-    return ent.get("bytes_per_launch")
+    for line in open(p):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 3 and cells[0] == kclass and cells[1] == source_digest(kclass):
+            try:
+                return float(cells[2])
+            except ValueError:
+                return None
+    return None
 
 
 # ------------------------------------------------------------------ CPU oracle timings

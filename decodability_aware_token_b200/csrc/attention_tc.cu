@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_const
     const int n_chunks = n_prefix_chunks + 1;
     // split-KV: this CTA walks chunks [c_begin, c_end) of the unit's n_chunks
     const int pieces = a.pieces;  // grid.y = Hkv * pieces
-    const int cpp = (n_chunks + pieces - 1) / pieces;
+    const int cpp = (n_chunks + pieces - 1) / pieces;  // chunks per piece
     const int piece = blockIdx.y / a.Hkv;
     const int c_begin = piece * cpp, c_end = min(n_chunks, c_begin + cpp);
     if (c_begin >= c_end) return;
@@ -183,11 +183,6 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_const
         pt_s[i] = a.page_table[(size_t)u.b * a.max_pages + i];
     const int32_t* pt = pt_cached ? pt_s : a.page_table + (size_t)u.b * a.max_pages;
 
-    // zero the ring once: skipped pages and short blocks then leave finite values behind masked keys
-    {
-        uint4* z = reinterpret_cast<uint4*>(kv);
-        for (int i = threadIdx.x; i < kStages * kStageBytes / 16; i += 128) z[i] = make_uint4(0, 0, 0, 0);
-    }
     if (threadIdx.x == 0) {
         for (int s2 = 0; s2 < kStages; ++s2) mbar_init(&full_bar[s2], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -195,7 +190,6 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_const
     __syncthreads();
     int issued = 0;  // chunks whose copies thread 0 has issued
     if (threadIdx.x == 0) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // zeros before the TMA writes
         for (int i = 0; i < kStages - 1 && c_begin + i < c_end; ++i) {
             valid_s[i] = issue_chunk(a, u, &pool_map, &ibc_map, kv + i * kStageBytes, &full_bar[i], c_begin + i,
                                      n_prefix_chunks, pt);
@@ -242,6 +236,7 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_const
         const int st = i % kStages;
         if (threadIdx.x == 0 && ci + kStages - 1 < c_end) {
             const int sn = (i + kStages - 1) % kStages;  // stage of chunk ci - 1: free since the last sync
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // V rows zeroed below, before TMA
             valid_s[sn] = issue_chunk(a, u, &pool_map, &ibc_map, kv + sn * kStageBytes, &full_bar[sn],
                                       ci + kStages - 1, n_prefix_chunks, pt);
             ++issued;
@@ -254,6 +249,15 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_const
         const uint64_t vmask = valid_s[st];
         const uint32_t kbase = smem_u32(kv + st * kStageBytes);
         const uint32_t vbase = kbase + 2 * kHalf;
+        if (vmask != ~0ull) {  // block-uniform: V rows of keys the copies left unfilled (skipped pages,
+                               // a short block) may hold stale bits; P is 0 there, so make V 0 too
+            uint8_t* vb = kv + st * kStageBytes + 2 * kHalf;
+            for (int t = threadIdx.x; t < kChunk * 16; t += 128) {
+                const int r = t >> 4, c = t & 15;
+                if (!((vmask >> r) & 1ull)) *reinterpret_cast<uint4*>(vb + swz(r, c)) = make_uint4(0, 0, 0, 0);
+            }
+            __syncthreads();
+        }
         // S = Q K^T over this warp's key slice: keys_per_warp / 8 n-tiles (up to 8)
         float s[8][4];
         const int n_nt = keys_per_warp / 8;
@@ -546,7 +550,8 @@ int attention_pieces(int units, int max_chunks) {
     // request walk sets the kernel's duration; capped by the split scratch
     constexpr int kTargetCtas = 4 * 148;
     // with at least one unit per SM the walks are long-lived streams already: splitting them only adds
-    // start-up and merge cost per piece (measured), so only few-unit launches are split
+    // start-up and merge cost per piece (measured, also with length-aware pieces), so only few-unit
+    // launches are split
     if (units <= 0 || units >= 148 || units > kAttnSplitCap) return 1;
     int p = (kTargetCtas + units - 1) / units;
     if (p > max_chunks) p = max_chunks;
