@@ -247,6 +247,31 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ replicas (one process per GPU)
+# Requests are independent, so N GPUs run N replicas, each on its own batch of the workload (no
+# collective on the data path); the ranks meet only to time the job: the slowest rank's device time
+# and the sum of the tokens all ranks decoded.
+def rank_seed(base: int, rank: int) -> int:
+    """Seed of rank `rank`'s requests (same shapes and distributions, different draws)."""
+    return base + 7919 * rank
+
+
+def reduce_over_ranks(elapsed_ms: float, decoded: float, world: int, device) -> tuple[float, float]:
+    """(max over ranks of elapsed_ms, sum over ranks of decoded); a collective only when world > 1."""
+    import torch.distributed as dist
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    tk = torch.tensor([decoded], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(tk, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(tk.item())
+
+
+def whole_job_rate(total_units: float, max_ms: float) -> float:
+    """Units all ranks processed per second of the slowest rank's time."""
+    return total_units / (max_ms / 1e3) if max_ms > 0 else 0.0
+
+
 # ------------------------------------------------------------------ the GPU arm
 def main():
     args = parse()
@@ -270,7 +295,7 @@ def main():
             dist.barrier()
 
     base = fs.SEEDS.get(args.workload, 1234)
-    case = make_workload(args, base + 7919 * rank, dev)    # this rank's requests
+    case = make_workload(args, rank_seed(base, rank), dev)    # this rank's requests
     w, shp = case.work, case.shape
     N, B = w.n_requests, w.block
     params = StepParams(w.tau, w.k_min, w.k_max, w.conf_threshold, w.alpha, w.forced_keep_frac)
@@ -385,13 +410,8 @@ def main():
     clocks = sampler.summary(tw0, tw1)
     elapsed = ev0.elapsed_time(ev1)
     decoded = int((out.decoded_ids >= 0).sum()) * K     # every step repeats the same (deterministic) work
-    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-    tk = torch.tensor([decoded], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dist.all_reduce(tk, op=dist.ReduceOp.SUM)
-    max_ms, total_decoded = float(t.item()), float(tk.item())
-    value = total_decoded / (max_ms / 1e3)
+    max_ms, total_decoded = reduce_over_ranks(elapsed, decoded, world, dev)
+    value = whole_job_rate(total_decoded, max_ms)
     del graph, graph_prof
 
     # ---- end to end through the public API (eager calls) with pinned host buffers
@@ -417,12 +437,8 @@ def main():
         torch.cuda.synchronize(dev)
         e_ms = e0.elapsed_time(e1)
         e_dec = int((out_h.decoded_ids >= 0).sum()) * K
-        te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        tke = torch.tensor([e_dec], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-            dist.all_reduce(tke, op=dist.ReduceOp.SUM)
-        e2e = {"value": float(tke.item()) / (float(te.item()) / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e_max_ms, e_total = reduce_over_ranks(e_ms, e_dec, world, dev)
+        e2e = {"value": whole_job_rate(e_total, e_max_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
 
     # ---- roofline of the dominant kernel class
