@@ -35,6 +35,7 @@ struct focus_ctx {
     void *h, *q, *o, *act;
     int32_t *row_req, *row_pos, *row_src, *n_rows, *lm_arg;
     double* inv_freq;
+    float2* rope_tab;     // bf16 path: [rope_positions][head_dim / 2] (cos, sin)
     int* err;
     float *att_part_o, *att_part_ml, *att_sb;
     int* att_counters;
@@ -92,6 +93,9 @@ int imp_tiles(const focus_model_cfg* c, const focus_limits* l) {
     return c->dtype == FOCUS_DTYPE_BF16 ? attention_q_tiles(l->max_block, c->n_q_heads / c->n_kv_heads) : 1;
 }
 
+// rotary positions a step can reach: the longest prefix (largest page size) plus the block
+size_t rope_positions(const focus_limits* l) { return (size_t)l->max_pages_per_req * 64 + l->max_block; }
+
 Layout plan(const focus_model_cfg* c, const focus_limits* l) {
     const size_t elt = c->dtype == FOCUS_DTYPE_BF16 ? 2 : 4;
     const size_t rows_full = (size_t)l->max_requests * l->max_block;
@@ -123,10 +127,11 @@ Layout plan(const focus_model_cfg* c, const focus_limits* l) {
         split * (size_t)kAttnSplitCap * 4,                  // 20 arrival counters
         (size_t)kGemmCounters * 4,                          // 21 split-K GEMM tile counters
         rows_c * 4, rows_c * 4,                             // 22-23 per-row confidence / top id
+        split * rope_positions(l) * (size_t)c->head_dim / 2 * 8,  // 24 RoPE (cos, sin) table
     };
     Layout lay{};
     size_t at = 0;
-    for (int i = 0; i < 24; ++i) {
+    for (int i = 0; i < 25; ++i) {
         lay.off[i] = at;
         at = align_up(at + sizes[i], 1024);
     }
@@ -201,7 +206,8 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
         g.lm_max = c->lm_max; g.lm_sum = c->lm_sum; g.lm_arg = c->lm_arg;
         g.counters = c->gemm_counters; g.resid = resid; g.q_out = c->q; g.ibc = in->ibc;
         g.row_req = compact ? c->row_req : nullptr; g.row_pos = compact ? c->row_pos : nullptr;
-        g.prefix_len = in->prefix_len; g.inv_freq = c->inv_freq; g.max_prefix = max_prefix; g.block = B;
+        g.prefix_len = in->prefix_len; g.inv_freq = c->inv_freq; g.rope_tab = c->rope_tab; g.max_prefix = max_prefix;
+        g.block = B;
         g.n_layers = dm.L; g.layer = layer; g.Hq = dm.Hq; g.Hkv = dm.Hkv; g.err = c->err;
         run(kclass, [&] {
             if (tc) return tc_gemm(c->tc, epi, wid, g, s);
@@ -426,6 +432,7 @@ int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_l
     c->lm_sum = reinterpret_cast<float*>(base + lay.off[13]);
     c->lm_arg = reinterpret_cast<int32_t*>(base + lay.off[14]);
     c->inv_freq = reinterpret_cast<double*>(base + lay.off[15]);
+    c->rope_tab = reinterpret_cast<float2*>(base + lay.off[24]);
     c->err = reinterpret_cast<int*>(base + lay.off[16]);
     c->att_part_o = reinterpret_cast<float*>(base + lay.off[17]);
     c->att_part_ml = reinterpret_cast<float*>(base + lay.off[18]);
@@ -444,6 +451,17 @@ int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_l
     for (int i = 0; i < cfg->head_dim / 2; ++i)
         inv[i] = pow((double)cfg->rope_theta, -2.0 * i / (double)cfg->head_dim);
     int rc = FOCUS_OK;
+    if (cfg->dtype == FOCUS_DTYPE_BF16) {
+        const size_t npos = rope_positions(lim), half = (size_t)cfg->head_dim / 2;
+        std::vector<float2> tab(npos * half);
+        for (size_t pos = 0; pos < npos; ++pos)
+            for (size_t i = 0; i < half; ++i) {
+                const double ang = (double)pos * inv[i];
+                tab[pos * half + i] = make_float2((float)cos(ang), (float)sin(ang));
+            }
+        if (cudaMemcpy(c->rope_tab, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess)
+            rc = FOCUS_ERR_CUDA;
+    }
     if (cudaMemcpy(c->inv_freq, inv.data(), inv.size() * sizeof(double), cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemset(c->err, 0, sizeof(int)) != cudaSuccess || cudaMemset(c->n_rows, 0, sizeof(int)) != cudaSuccess ||
         cudaMemset(c->gemm_counters, 0, (size_t)kGemmCounters * 4) != cudaSuccess ||

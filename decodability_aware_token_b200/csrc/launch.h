@@ -157,6 +157,7 @@ struct GemmArgs {
     const int32_t* row_pos;
     const int32_t* prefix_len;
     const double* inv_freq;     // [d / 2] RoPE frequencies
+    const float2* rope_tab;     // tensor-core epilogues: [positions][d / 2] (cos, sin) of pos * inv_freq
     int max_prefix, block, n_layers, layer, Hq, Hkv;
     int* err;
 };

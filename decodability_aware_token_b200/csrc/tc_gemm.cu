@@ -105,6 +105,8 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
          set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_RESID>, Big::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_QKV>, Big::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL>, Small::SMEM) &&
+         set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_RESID>, Small::SMEM) &&
+         set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_QKV>, Small::SMEM) &&
          set_smem((const void*)tc_gemmt_kernel<EPI_RESID>, kTSmem) &&
          set_smem((const void*)tc_gemmt_kernel<EPI_QKV>, kTSmem) &&
          set_smem((const void*)tc_gemmt_kernel<EPI_SWIGLU>, kTSmem) &&
@@ -190,9 +192,13 @@ int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g0, cudaStream_t s) {
     GemmArgs g = g0;
     const bool small = g.M_bound <= kSmallRows;
     if (small && epi != EPI_PARTIAL) return tc_gemm_swapped(p, epi, g, s);
-    const CUtensorMap* a = g.A == p->h ? (small ? &p->map_h1 : &p->map_h)
-                         : g.A == p->o ? (small ? &p->map_o1 : &p->map_o)
-                                       : (small ? &p->map_act1 : &p->map_act);
+    // residual and QKV GEMMs whose 256-row tiles would leave SMs idle take 128-row tiles
+    const int n_tiles_big = (g.N + kBN - 1) / kBN;
+    const bool rows128 = small || ((epi == EPI_RESID || epi == EPI_QKV) &&
+                                   n_tiles_big * ((g.M_bound + Big::BM - 1) / Big::BM) < p->sms);
+    const CUtensorMap* a = g.A == p->h ? (rows128 ? &p->map_h1 : &p->map_h)
+                         : g.A == p->o ? (rows128 ? &p->map_o1 : &p->map_o)
+                                       : (rows128 ? &p->map_act1 : &p->map_act);
     const CUtensorMap* b = &p->wmap.find(g.B)->second;
     const CUtensorMap* b2 = epi == EPI_SWIGLU ? &p->wmap.find(g.B2)->second : b;
     int splits = (epi == EPI_PARTIAL || epi == EPI_RESID || epi == EPI_QKV) ? g.splits : 1;
@@ -203,13 +209,19 @@ int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g0, cudaStream_t s) {
         g.n_tiles = n_tiles;
         g.tile_n = kBN;
     }
-    const int bm = small ? Small::BM : Big::BM;
+    const int bm = rows128 ? Small::BM : Big::BM;
     dim3 grid(n_tiles, (g.M_bound + bm - 1) / bm, splits);
     (void)wid;
     const dim3 blk(192);
     if (small)  // EPI_PARTIAL
         return launched(launch_pdl(tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL>, grid, blk, Small::SMEM, s, 0, *a, *b, *b2,
                                    g, p->err));
+    if (rows128 && epi == EPI_RESID)
+        return launched(launch_pdl(tc_gemm_kernel<kBN, 1, kStages, EPI_RESID>, grid, blk, Small::SMEM, s, 0, *a, *b, *b2,
+                                   g, p->err));
+    if (rows128 && epi == EPI_QKV)
+        return launched(launch_pdl(tc_gemm_kernel<kBN, 1, kStages, EPI_QKV>, grid, blk, Small::SMEM, s, 0, *a, *b, *b2, g,
+                                   p->err));
     switch (epi) {
         case EPI_PARTIAL:
             return launched(launch_pdl(tc_gemm_kernel<kBN, 2, kStages, EPI_PARTIAL>, grid, blk, Big::SMEM, s, 0, *a, *b,

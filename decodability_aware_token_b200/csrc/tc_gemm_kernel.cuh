@@ -112,13 +112,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// RoPE angle of block position pos for pair i: reduced modulo 2 pi in double (two-term 2 pi), then a
-// float sincos on [-pi, pi].
-__device__ __forceinline__ void rope_cs(int pos, double inv_freq, float& cn, float& sn) {
-    const double ang = (double)pos * inv_freq;
-    const double k = rint(ang * 0.15915494309189535);
-    const double red = (ang - k * 6.283185307179586) - k * 2.4492935982947064e-16;
-    sincosf((float)red, &sn, &cn);
+// RoPE (cos, sin) of rotary position pos for pair i (head dim 128): a table the context fills once in
+// double precision, rounded to float (positions up to the longest prefix plus the block).
+__device__ __forceinline__ void rope_cs(const GemmArgs& g, int pos, int i, float& cn, float& sn) {
+    const float2 cs = __ldg(g.rope_tab + (size_t)pos * 64 + i);
+    cn = cs.x;
+    sn = cs.y;
 }
 
 // (request, block position, rotary position) of a GEMM row in the QKV epilogue
@@ -333,8 +332,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
                                 float a0 = lo[t], a1 = lo[t + 1], b0 = hi[t], b1 = hi[t + 1];
                                 if (rotate) {
                                     float c_0, s_0, c_1, s_1;
-                                    rope_cs(pos, g.inv_freq[c0 + t], c_0, s_0);
-                                    rope_cs(pos, g.inv_freq[c0 + t + 1], c_1, s_1);
+                                    rope_cs(g, pos, c0 + t, c_0, s_0);
+                                    rope_cs(g, pos, c0 + t + 1, c_1, s_1);
                                     a0 = lo[t] * c_0 - hi[t] * s_0;
                                     b0 = hi[t] * c_0 + lo[t] * s_0;
                                     a1 = lo[t + 1] * c_1 - hi[t + 1] * s_1;
@@ -470,7 +469,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
                                 if (head < g.Hq + g.Hkv) {
                                     const int i = (col + e) & 63;
                                     float cn, sn;
-                                    rope_cs(pos, g.inv_freq[i], cn, sn);
+                                    rope_cs(g, pos, i, cn, sn);
                                     o4[e] = col < 64 ? v[e] * cn - partner * sn : v[e] * cn + partner * sn;
                                 } else {
                                     o4[e] = v[e];
@@ -720,7 +719,6 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
         } else {
             // thread e finishes feature pair (fp, fp + 64) for the tokens of parity e / 64
             const int fp = e & 63;
-            const double inv = EPI == EPI_QKV ? g.inv_freq[fp] : 0.0;
             for (int t = t0 + (e >> 6); t < t1; t += 4) {
                 float lo_p[2][kTMaxSplits], hi_p[2][kTMaxSplits];
 #pragma unroll
@@ -754,7 +752,7 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
                         float lo = a, hi = bb;
                         if (head < g.Hq + g.Hkv) {
                             float cn, sn;
-                            rope_cs(pos, inv, cn, sn);
+                            rope_cs(g, pos, fp, cn, sn);
                             lo = a * cn - bb * sn;
                             hi = bb * cn + a * sn;
                         }
