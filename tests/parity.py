@@ -11,7 +11,8 @@ Rules (what is unique is compared exactly, what is not is checked for validity):
     storage alone causes (bf16-storage oracle minus float64 oracle, measured per quantity): deep
     random-weight stacks amplify bf16-level perturbations, so two equally valid bf16 evaluations that
     differ only in summation order already differ by about that drift (4.2% of RMS at 28 layers);
-    the RMS of the error must stay within frac x RMS regardless;
+    likewise the RMS of the error stays within frac x RMS plus twice the RMS of that drift (the
+    8B shape's 36 layers give confidences a bf16 drift of several % RMS);
   * kept set per request: identical wherever the oracle's delta gap at the top-k cut and its
     |delta - tau| both exceed the selection gate; otherwise the GPU set must still be a valid top-k of
     the oracle's deltas within that gate (and the test then re-runs the GPU with the oracle's set
@@ -59,8 +60,8 @@ def _rms(x):
     return float(np.sqrt(np.mean(x * x))) if x.size else 0.0
 
 
-def close(name, got, want, frac, report, allow=0.0):
-    """max|got - want| <= frac * RMS(want) + allow, and RMS(got - want) <= frac * RMS(want)."""
+def close(name, got, want, frac, report, allow=0.0, allow_rms=0.0):
+    """max|got - want| <= frac * RMS(want) + allow, and RMS(got - want) <= frac * RMS(want) + allow_rms."""
     got, want = np.asarray(got, np.float64), np.asarray(want, np.float64)
     assert got.shape == want.shape, f"{name}: shape {got.shape} vs {want.shape}"
     if got.size == 0:
@@ -68,10 +69,11 @@ def close(name, got, want, frac, report, allow=0.0):
     err = float(np.max(np.abs(got - want)))
     rms_err = _rms(got - want)
     scale = _rms(want)
-    report[name] = dict(max_abs=err, rms_err=rms_err, rms=scale, allow=allow)
+    report[name] = dict(max_abs=err, rms_err=rms_err, rms=scale, allow=allow, allow_rms=allow_rms)
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
     assert err <= frac * scale + allow, f"{name}: max-abs error {err:.3e} > {frac} x RMS {scale:.3e} + {allow:.3e}"
-    assert rms_err <= frac * scale, f"{name}: RMS error {rms_err:.3e} > {frac} x RMS {scale:.3e}"
+    assert rms_err <= frac * scale + allow_rms, \
+        f"{name}: RMS error {rms_err:.3e} > {frac} x RMS {scale:.3e} + {allow_rms:.3e}"
 
 
 def valid_selection(kept_gpu, delta, masked, params, sel_gate, B):
@@ -118,14 +120,19 @@ def derived_logit_gate(case, frac):
 
 
 def drift_allowance(ora: fo.OracleResult, ora_exact: fo.OracleResult) -> dict:
-    """Twice the max-abs change that bf16 storage alone makes (same kept sets on both oracles)."""
+    """Twice the change that bf16 storage alone makes (same kept sets on both oracles): its max-abs for the
+    max-abs bounds, its RMS ("<name>_rms") for the RMS bounds."""
     mk = np.zeros_like(ora.conf, dtype=bool)
     for b in range(ora.keep_count.shape[0]):
         mk[b, : ora.keep_count[b]] = True
     d = lambda a, b: 2.0 * float(np.abs(a - b).max()) if a.size else 0.0
-    return {"importance": d(ora.importance, ora_exact.importance), "hidden": d(ora.hidden, ora_exact.hidden),
-            "conf": d(ora.conf[mk], ora_exact.conf[mk]), "ibc": d(ora.ibc, ora_exact.ibc),
-            "hidden_rel": d(ora.hidden, ora_exact.hidden) / max(_rms(ora_exact.hidden), 1e-30)}
+    r = lambda a, b: 2.0 * _rms(a - b) if a.size else 0.0
+    out = {"importance": d(ora.importance, ora_exact.importance), "hidden": d(ora.hidden, ora_exact.hidden),
+           "conf": d(ora.conf[mk], ora_exact.conf[mk]), "ibc": d(ora.ibc, ora_exact.ibc),
+           "hidden_rel": d(ora.hidden, ora_exact.hidden) / max(_rms(ora_exact.hidden), 1e-30)}
+    out.update(importance_rms=r(ora.importance, ora_exact.importance), hidden_rms=r(ora.hidden, ora_exact.hidden),
+               conf_rms=r(ora.conf[mk], ora_exact.conf[mk]), ibc_rms=r(ora.ibc, ora_exact.ibc))
+    return out
 
 
 def compare(case, params: dict, ora: fo.OracleResult, gpu: dict, tol: Tol, ibc_in, check_selection=True,
@@ -138,7 +145,8 @@ def compare(case, params: dict, ora: fo.OracleResult, gpu: dict, tol: Tol, ibc_i
         derived_logit_gate(case, tol.frac + allow.get("hidden_rel", 0.0))
     lc_gate = tol.log_conf if tol.log_conf is not None else 2 * logit_gate
     report["logit_gate"] = logit_gate
-    close("importance", gpu["importance"], ora.importance, tol.frac, report, allow.get("importance", 0.0))
+    close("importance", gpu["importance"], ora.importance, tol.frac, report, allow.get("importance", 0.0),
+          allow.get("importance_rms", 0.0))
     kc = _np(gpu["keep_count"])
     ret = _np(gpu["retained_idx"])
     masked0 = _np(case.batch["mask"]).astype(bool)
@@ -161,12 +169,13 @@ def compare(case, params: dict, ora: fo.OracleResult, gpu: dict, tol: Tol, ibc_i
     if flipped:
         return report, flipped
     # downstream: identical kept sets from here on
-    close("hidden", _np(gpu["hidden"])[: off[-1]], ora.hidden, tol.frac, report, allow.get("hidden", 0.0))
+    close("hidden", _np(gpu["hidden"])[: off[-1]], ora.hidden, tol.frac, report, allow.get("hidden", 0.0),
+          allow.get("hidden_rms", 0.0))
     conf_g, top_g = _np(gpu["conf"]), _np(gpu["top_id"])
     mask_k = np.zeros_like(conf_g, dtype=bool)
     for b in range(N):
         mask_k[b, : kc[b]] = True
-    close("conf", conf_g[mask_k], ora.conf[mask_k], tol.frac, report, allow.get("conf", 0.0))
+    close("conf", conf_g[mask_k], ora.conf[mask_k], tol.frac, report, allow.get("conf", 0.0), allow.get("conf_rms", 0.0))
     assert np.all(conf_g[~mask_k] == 0) and np.all(top_g[~mask_k] == -1), "unused conf / top slots"
     n_tie_ids = 0
     for b in range(N):
@@ -212,6 +221,7 @@ def compare(case, params: dict, ora: fo.OracleResult, gpu: dict, tol: Tol, ibc_i
     for b in range(N):
         written[b, 2:, ora.retained_idx[b, : ora.keep_count[b]]] = True
     w_idx = np.broadcast_to(written[:, :, None, None, :, None], ibc_g.shape)
-    close("ibc_written", ibc_g[w_idx], ora.ibc[w_idx], tol.frac, report, allow.get("ibc", 0.0))
+    close("ibc_written", ibc_g[w_idx], ora.ibc[w_idx], tol.frac, report, allow.get("ibc", 0.0),
+          allow.get("ibc_rms", 0.0))
     assert np.array_equal(ibc_g[~w_idx], ibc0[~w_idx]), "an evicted position's cache entry changed"
     return report, []

@@ -4,6 +4,7 @@ Small cases span several GEMM / attention tiles and ragged tails; the full-size 
 checked on sampled requests (requests are independent, so the oracle can run a subset).
 """
 import dataclasses
+import gc
 
 import numpy as np
 import pytest
@@ -203,6 +204,7 @@ def test_step_replays_from_cuda_graph():
 
 # ---------------------------------------------------------------- full-size workloads, sampled requests
 @pytest.mark.slow
+@pytest.mark.usefixtures("free_device_memory")
 def test_sdar_1p7b_n32_b32_sampled():
     case = fs.make_case("sdar1.7b_n32_b32", device="cuda:0")
     host = fs.Case(case.shape, case.work, {k: ([t.cpu() for t in v] if isinstance(v, list) else v.cpu())
@@ -211,4 +213,62 @@ def test_sdar_1p7b_n32_b32_sampled():
     p = step_params(case.work)
     gpu = run_gpu(host, p, case.model)
     rep = check(host, p, requests=[0, 13, 31], gpu=gpu)
+    print(rep)
+
+
+@pytest.fixture
+def free_device_memory():
+    """The full-size cases hold tens of GB on the device: release them before and after each test."""
+    _models.clear()
+    gc.collect()
+    torch.cuda.empty_cache()
+    yield
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def _sampled_check(case, requests, params=None):
+    """Full-size case on the GPU (model, pages and cache stay on the device); the oracle runs only the
+    sampled requests (requests are independent) and reads their pages from the device."""
+    p = params or step_params(case.work)
+    gpu = run_gpu(case, p, case.model)
+    host = fs.Case(case.shape, case.work, case.model, {k: (v if k == "kv_pool" else v.cpu()) for k, v in case.batch.items()},
+                   case.seed)
+    rep = check(host, p, requests=requests, gpu=gpu)
+    del gpu, host
+    return rep
+
+
+@pytest.mark.slow
+@pytest.mark.usefixtures("free_device_memory")
+def test_sdar_1p7b_n128_lognormal_sampled():
+    # 128 ragged requests, prefixes log-normal (median 600, clipped to 64..4096), k_max 12: the kept rows
+    # exceed the few-row GEMM bound, so the later layers run on the 256-row tensor-core tiles
+    case = fs.make_case("sdar1.7b_n128_b32", device="cuda:0")
+    plen = case.batch["prefix_len"].cpu()
+    longest = int(torch.argmax(plen))
+    rep = _sampled_check(case, sorted({0, longest, 127}))
+    del case
+    print(rep)
+
+
+@pytest.mark.slow
+@pytest.mark.usefixtures("free_device_memory")
+def test_sdar_8b_n256_b64_sampled():
+    # 8B shape (hidden 4096, 32 / 8 heads: four query heads per KV head), block 64, k_max 16
+    case = fs.make_case("sdar8b_n256_b64", device="cuda:0")
+    rep = _sampled_check(case, [0, 255])
+    del case
+    print(rep)
+
+
+@pytest.mark.slow
+@pytest.mark.usefixtures("free_device_memory")
+@pytest.mark.parametrize("n,block,frac", [(64, 64, 0.5), (32, 16, 0.25), (128, 32, 0.1)])
+def test_kernel_sweep_points_sampled(n, block, frac):
+    # sweep points on the 1.7B shape with a forced keep fraction (prefixes U[256, 4096])
+    case = fs.make_case("sweep", seed=fs.SEEDS["sweep"], device="cuda:0", shape=fs.MODEL_SHAPES["sdar1.7b"],
+                        work=fs.sweep_workload(n, block, frac))
+    rep = _sampled_check(case, [0, n - 1])
+    del case
     print(rep)
