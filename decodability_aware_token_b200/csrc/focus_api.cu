@@ -39,7 +39,6 @@ struct focus_ctx {
     int* err;
     float *att_part_o, *att_part_ml, *att_sb;
     int* att_counters;
-    int* gemm_counters;
     float* row_conf;
     int32_t* row_top;
     size_t part_rows;     // rows of the partial-sum buffer
@@ -125,13 +124,12 @@ Layout plan(const focus_model_cfg* c, const focus_limits* l) {
         split * (size_t)kAttnSplitCap * 64 * 2 * 4,         // 18 partial row max / denominator
         split * (size_t)kAttnSplitCap * 64 * 64 * 4,        // 19 raw block scores
         split * (size_t)kAttnSplitCap * 4,                  // 20 arrival counters
-        (size_t)kGemmCounters * 4,                          // 21 split-K GEMM tile counters
-        rows_c * 4, rows_c * 4,                             // 22-23 per-row confidence / top id
-        split * rope_positions(l) * (size_t)c->head_dim / 2 * 8,  // 24 RoPE (cos, sin) table
+        rows_c * 4, rows_c * 4,                             // 21-22 per-row confidence / top id
+        split * rope_positions(l) * (size_t)c->head_dim / 2 * 8,  // 23 RoPE (cos, sin) table
     };
     Layout lay{};
     size_t at = 0;
-    for (int i = 0; i < 25; ++i) {
+    for (int i = 0; i < 24; ++i) {
         lay.off[i] = at;
         at = align_up(at + sizes[i], 1024);
     }
@@ -198,19 +196,19 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
         }
     };
     auto gemm = [&](int kclass, Epi epi, const void* A, const void* Bw, const void* B2, int Mb, const int32_t* Md,
-                    int Nn, int K, int splits, int wid, void* act_out, float* resid = nullptr, int layer = 0,
+                    int Nn, int K, int splits, void* act_out, float* resid = nullptr, int layer = 0,
                     bool compact = false) {
         GemmArgs g{};
         g.A = A; g.B = Bw; g.B2 = B2; g.M_bound = Mb; g.M_dev = Md; g.N = Nn; g.K = K; g.splits = splits;
         g.part = c->part; g.split_stride = stride; g.act = act_out;
         g.lm_max = c->lm_max; g.lm_sum = c->lm_sum; g.lm_arg = c->lm_arg;
-        g.counters = c->gemm_counters; g.resid = resid; g.q_out = c->q; g.ibc = in->ibc;
+        g.resid = resid; g.q_out = c->q; g.ibc = in->ibc;
         g.row_req = compact ? c->row_req : nullptr; g.row_pos = compact ? c->row_pos : nullptr;
         g.prefix_len = in->prefix_len; g.inv_freq = c->inv_freq; g.rope_tab = c->rope_tab; g.max_prefix = max_prefix;
         g.block = B;
         g.n_layers = dm.L; g.layer = layer; g.Hq = dm.Hq; g.Hkv = dm.Hkv; g.err = c->err;
         run(kclass, [&] {
-            if (tc) return tc_gemm(c->tc, epi, wid, g, s);
+            if (tc) return tc_gemm(c->tc, epi, g, s);
             g.n_tiles = (Nn + kSimtTileN - 1) / kSimtTileN;
             g.tile_n = kSimtTileN;
             return launch_gemm_simt<T>(epi, g, s);
@@ -235,16 +233,13 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
                                     c->x_full, h, c->err, s);
     });
     // tensor-core path: the GEMM epilogues apply RoPE + the cache write (QKV) and the residual adds
-    // (O, down) themselves, reducing split-K partials in the GEMM; the row kernels only normalise
-    if (tc) FOCUS_CUDA_TRY(cudaMemsetAsync(c->gemm_counters, 0, (size_t)kGemmCounters * 4, s));
+    // (O, down) themselves, reducing any split-K slices inside the GEMM; the row kernels only normalise
     // ---- layers 0 and 1: full block, importance at both
     for (int l = 0; l < 2; ++l) {
         if (tc) {
-            gemm(FOCUS_K_GEMM_FULL_QKV, EPI_QKV, c->h, c->wqkv[l], nullptr, rows_full, nullptr, dm.qkv, dm.D, 1,
-                 W_QKV, nullptr, nullptr, l, false);
+            gemm(FOCUS_K_GEMM_FULL_QKV, EPI_QKV, c->h, c->wqkv[l], nullptr, rows_full, nullptr, dm.qkv, dm.D, 1, nullptr, nullptr, l, false);
         } else {
-            gemm(FOCUS_K_GEMM_FULL_QKV, EPI_PARTIAL, c->h, c->wqkv[l], nullptr, rows_full, nullptr, dm.qkv, dm.D, 1,
-                 W_QKV, nullptr);
+            gemm(FOCUS_K_GEMM_FULL_QKV, EPI_PARTIAL, c->h, c->wqkv[l], nullptr, rows_full, nullptr, dm.qkv, dm.D, 1, nullptr);
             run(FOCUS_K_QKV_FINALIZE, [&] {
                 return launch_qkv_finalize<T>(c->part, 1, stride, full, in->prefix_len, max_prefix, c->inv_freq, dm,
                                               l, q, ibc, c->err, s);
@@ -257,15 +252,14 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
         run(FOCUS_K_ATTN_SCORE, [&] { return attention(at, qt_full); });
         const int nsp_full = tc ? 0 : 1;  // partial slices the norm kernels still add (CUDA-core path)
         gemm(FOCUS_K_GEMM_FULL_O, tc ? EPI_RESID : EPI_PARTIAL, c->o, c->wo[l], nullptr, rows_full, nullptr, dm.D,
-             dm.Hq * dm.d, 1, W_O, nullptr, c->x_full, l, false);
+             dm.Hq * dm.d, 1, nullptr, c->x_full, l, false);
         run(FOCUS_K_ROW_NORM, [&] {
             return launch_residual_norm<T>(c->x_full, nullptr, nullptr, rows_full, c->part, nsp_full, stride, c->x_full,
                                            W(c->mlp_norm[l]), dm.eps, dm.D, h, s);
         });
-        gemm(FOCUS_K_GEMM_FULL_GATEUP, EPI_SWIGLU, c->h, c->wgate[l], c->wup[l], rows_full, nullptr, dm.F, dm.D, 1,
-             W_GATEUP, c->act);
+        gemm(FOCUS_K_GEMM_FULL_GATEUP, EPI_SWIGLU, c->h, c->wgate[l], c->wup[l], rows_full, nullptr, dm.F, dm.D, 1, c->act);
         gemm(FOCUS_K_GEMM_FULL_DOWN, tc ? EPI_RESID : EPI_PARTIAL, c->act, c->wdown[l], nullptr, rows_full, nullptr,
-             dm.D, dm.F, 1, W_DOWN, nullptr, c->x_full, l, false);
+             dm.D, dm.F, 1, nullptr, c->x_full, l, false);
         if (l == 0)
             run(FOCUS_K_ROW_NORM, [&] {
                 return launch_residual_norm<T>(c->x_full, nullptr, nullptr, rows_full, c->part, nsp_full, stride,
@@ -293,11 +287,10 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
     const int sp_qkv = 1, sp_o = 1, sp_dn = 1;
     for (int l = 2; l < dm.L; ++l) {
         if (tc) {
-            gemm(FOCUS_K_GEMM_QKV, EPI_QKV, c->h, c->wqkv[l], nullptr, R_bound, c->n_rows, dm.qkv, dm.D, sp_qkv, W_QKV,
+            gemm(FOCUS_K_GEMM_QKV, EPI_QKV, c->h, c->wqkv[l], nullptr, R_bound, c->n_rows, dm.qkv, dm.D, sp_qkv,
                  nullptr, nullptr, l, true);
         } else {
-            gemm(FOCUS_K_GEMM_QKV, EPI_PARTIAL, c->h, c->wqkv[l], nullptr, R_bound, c->n_rows, dm.qkv, dm.D, sp_qkv,
-                 W_QKV, nullptr);
+            gemm(FOCUS_K_GEMM_QKV, EPI_PARTIAL, c->h, c->wqkv[l], nullptr, R_bound, c->n_rows, dm.qkv, dm.D, sp_qkv, nullptr);
             run(FOCUS_K_QKV_FINALIZE, [&] {
                 return launch_qkv_finalize<T>(c->part, sp_qkv, stride, comp, in->prefix_len, max_prefix, c->inv_freq,
                                               dm, l, q, ibc, c->err, s);
@@ -309,15 +302,14 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
         at.pieces = pieces_kept;
         run(FOCUS_K_ATTN_RAGGED, [&] { return attention(at, qt_kept); });
         gemm(FOCUS_K_GEMM_O, tc ? EPI_RESID : EPI_PARTIAL, c->o, c->wo[l], nullptr, R_bound, c->n_rows, dm.D,
-             dm.Hq * dm.d, sp_o, W_O, nullptr, c->x_c, l, true);
+             dm.Hq * dm.d, sp_o, nullptr, c->x_c, l, true);
         run(FOCUS_K_ROW_NORM, [&] {
             return launch_residual_norm<T>(c->x_c, nullptr, c->n_rows, R_bound, c->part, tc ? 0 : sp_o, stride, c->x_c,
                                            W(c->mlp_norm[l]), dm.eps, dm.D, h, s);
         });
-        gemm(FOCUS_K_GEMM_GATEUP, EPI_SWIGLU, c->h, c->wgate[l], c->wup[l], R_bound, c->n_rows, dm.F, dm.D, 1,
-             W_GATEUP, c->act);
+        gemm(FOCUS_K_GEMM_GATEUP, EPI_SWIGLU, c->h, c->wgate[l], c->wup[l], R_bound, c->n_rows, dm.F, dm.D, 1, c->act);
         gemm(FOCUS_K_GEMM_DOWN, tc ? EPI_RESID : EPI_PARTIAL, c->act, c->wdown[l], nullptr, R_bound, c->n_rows, dm.D,
-             dm.F, sp_dn, W_DOWN, nullptr, c->x_c, l, true);
+             dm.F, sp_dn, nullptr, c->x_c, l, true);
         const void* gn = l + 1 < dm.L ? c->attn_norm[l + 1] : c->final_norm;
         run(FOCUS_K_ROW_NORM, [&] {
             return launch_residual_norm<T>(c->x_c, nullptr, c->n_rows, R_bound, c->part, tc ? 0 : sp_dn, stride, c->x_c,
@@ -325,7 +317,7 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
         });
     }
     // ---- LM head (fused max / sum-exp / argmax per vocabulary tile), combine, decode
-    gemm(FOCUS_K_GEMM_LMHEAD, EPI_LMHEAD, c->h, c->lm_head, nullptr, R_bound, c->n_rows, dm.V, dm.D, 1, W_LM, nullptr);
+    gemm(FOCUS_K_GEMM_LMHEAD, EPI_LMHEAD, c->h, c->lm_head, nullptr, R_bound, c->n_rows, dm.V, dm.D, 1, nullptr);
     DecodeArgs da{};
     da.lm_max = c->lm_max; da.lm_sum = c->lm_sum; da.lm_arg = c->lm_arg;
     da.n_tiles = tc ? tc_lm_tiles(c->tc) : (dm.V + kSimtTileN - 1) / kSimtTileN;
@@ -432,15 +424,14 @@ int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_l
     c->lm_sum = reinterpret_cast<float*>(base + lay.off[13]);
     c->lm_arg = reinterpret_cast<int32_t*>(base + lay.off[14]);
     c->inv_freq = reinterpret_cast<double*>(base + lay.off[15]);
-    c->rope_tab = reinterpret_cast<float2*>(base + lay.off[24]);
+    c->rope_tab = reinterpret_cast<float2*>(base + lay.off[23]);
     c->err = reinterpret_cast<int*>(base + lay.off[16]);
     c->att_part_o = reinterpret_cast<float*>(base + lay.off[17]);
     c->att_part_ml = reinterpret_cast<float*>(base + lay.off[18]);
     c->att_sb = reinterpret_cast<float*>(base + lay.off[19]);
     c->att_counters = reinterpret_cast<int*>(base + lay.off[20]);
-    c->gemm_counters = reinterpret_cast<int*>(base + lay.off[21]);
-    c->row_conf = reinterpret_cast<float*>(base + lay.off[22]);
-    c->row_top = reinterpret_cast<int32_t*>(base + lay.off[23]);
+    c->row_conf = reinterpret_cast<float*>(base + lay.off[21]);
+    c->row_top = reinterpret_cast<int32_t*>(base + lay.off[22]);
     const size_t rows_full = (size_t)lim->max_requests * lim->max_block;
     const size_t rows_c = (size_t)lim->max_requests * lim->max_keep;
     c->part_rows = rows_full > kMaxSplits * rows_c ? rows_full : kMaxSplits * rows_c;
@@ -464,7 +455,6 @@ int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_l
     }
     if (cudaMemcpy(c->inv_freq, inv.data(), inv.size() * sizeof(double), cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemset(c->err, 0, sizeof(int)) != cudaSuccess || cudaMemset(c->n_rows, 0, sizeof(int)) != cudaSuccess ||
-        cudaMemset(c->gemm_counters, 0, (size_t)kGemmCounters * 4) != cudaSuccess ||
         (cfg->dtype == FOCUS_DTYPE_BF16 &&
          cudaMemset(c->att_counters, 0, (size_t)kAttnSplitCap * 4) != cudaSuccess))
         rc = FOCUS_ERR_CUDA;

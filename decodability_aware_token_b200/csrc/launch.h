@@ -147,9 +147,7 @@ struct GemmArgs {
     int32_t* lm_arg;
     int n_tiles;
     int tile_n;                 // EPI_LMHEAD: columns per stats tile
-    // tcgen05 fused epilogues (split K: every split writes its partial tile to `part`, and the last split
-    // CTA of each output tile -- counted in `counters`, zero between launches -- sums them in split order)
-    int* counters;
+    // tcgen05 fused epilogues
     float* resid;               // EPI_RESID: [rows, N] float32 residual stream, resid += A B^T
     void* q_out;                // EPI_QKV: [rows, Hq d] rotated queries (bf16)
     void* ibc;                  // EPI_QKV: intra-block KV cache [N, L, 2, Hkv, B, d]: rotated K and V at (b, j)
@@ -162,7 +160,6 @@ struct GemmArgs {
     int* err;
 };
 template <typename T> int launch_gemm_simt(Epi epi, const GemmArgs& g, cudaStream_t s);
-constexpr int kGemmCounters = 1024;  // arrival counters: output tiles of one split-K GEMM launch
 constexpr int kSimtTileN = 64;
 
 // ---- LM-head combine + threshold decode (decode.cu) ------------------------------

@@ -1,6 +1,5 @@
 // bf16 GEMM C = A B^T on the 5th-generation tensor cores (tcgen05.mma, accumulators in TMEM,
 // operands staged by TMA), with the step's fused epilogues:
-//   EPI_PARTIAL: float32 partial sums of one split-K slice -> part[split][m][n]
 //   EPI_SWIGLU:  the B tile is BN/2 gate rows followed by BN/2 up rows; writes silu(g) * u (bf16)
 //   EPI_LMHEAD:  per row and vocabulary tile: max logit, sum exp(z - max), first argmax (no logits in HBM)
 //   EPI_RESID:   resid += A B^T (float32 residual stream)
@@ -99,12 +98,10 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
         return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
                max_shared_carveout(fn);
     };
-    ok = set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_PARTIAL>, Big::SMEM) &&
-         set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_SWIGLU>, Big::SMEM) &&
+    ok = set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_SWIGLU>, Big::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_LMHEAD>, Big::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_RESID>, Big::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 2, kStages, EPI_QKV>, Big::SMEM) &&
-         set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL>, Small::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_RESID>, Small::SMEM) &&
          set_smem((const void*)tc_gemm_kernel<kBN, 1, kStages, EPI_QKV>, Small::SMEM) &&
          set_smem((const void*)tc_gemmt_kernel<EPI_RESID>, kTSmem) &&
@@ -187,35 +184,27 @@ int tc_gemm_swapped(TcPlan* p, Epi epi, GemmArgs g, cudaStream_t s) {
 
 }  // namespace
 
-int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g0, cudaStream_t s) {
+int tc_gemm(TcPlan* p, Epi epi, const GemmArgs& g0, cudaStream_t s) {
     if (g0.M_bound <= 0) return 0;
+    if (epi == EPI_PARTIAL) return -1;  // partial sums are the CUDA-core path's; these kernels fuse their epilogues
     GemmArgs g = g0;
-    const bool small = g.M_bound <= kSmallRows;
-    if (small && epi != EPI_PARTIAL) return tc_gemm_swapped(p, epi, g, s);
+    if (g.M_bound <= kSmallRows) return tc_gemm_swapped(p, epi, g, s);
     // residual and QKV GEMMs whose 256-row tiles would leave SMs idle take 128-row tiles
     const int n_tiles_big = (g.N + kBN - 1) / kBN;
-    const bool rows128 = small || ((epi == EPI_RESID || epi == EPI_QKV) &&
-                                   n_tiles_big * ((g.M_bound + Big::BM - 1) / Big::BM) < p->sms);
+    const bool rows128 = (epi == EPI_RESID || epi == EPI_QKV) &&
+                         n_tiles_big * ((g.M_bound + Big::BM - 1) / Big::BM) < p->sms;
     const CUtensorMap* a = g.A == p->h ? (rows128 ? &p->map_h1 : &p->map_h)
                          : g.A == p->o ? (rows128 ? &p->map_o1 : &p->map_o)
                                        : (rows128 ? &p->map_act1 : &p->map_act);
     const CUtensorMap* b = &p->wmap.find(g.B)->second;
     const CUtensorMap* b2 = epi == EPI_SWIGLU ? &p->wmap.find(g.B2)->second : b;
-    int splits = (epi == EPI_PARTIAL || epi == EPI_RESID || epi == EPI_QKV) ? g.splits : 1;
-    if (splits > g.K / BK) splits = g.K / BK;  // every split slice gets at least one K block
-    if (splits < 1) splits = 1;
     const int n_tiles = epi == EPI_SWIGLU ? g.N / (kBN / 2) : (g.N + kBN - 1) / kBN;
     if (epi == EPI_LMHEAD) {
         g.n_tiles = n_tiles;
         g.tile_n = kBN;
     }
     const int bm = rows128 ? Small::BM : Big::BM;
-    dim3 grid(n_tiles, (g.M_bound + bm - 1) / bm, splits);
-    (void)wid;
-    const dim3 blk(192);
-    if (small)  // EPI_PARTIAL
-        return launched(launch_pdl(tc_gemm_kernel<kBN, 1, kStages, EPI_PARTIAL>, grid, blk, Small::SMEM, s, 0, *a, *b, *b2,
-                                   g, p->err));
+    const dim3 grid(n_tiles, (g.M_bound + bm - 1) / bm, 1), blk(192);
     if (rows128 && epi == EPI_RESID)
         return launched(launch_pdl(tc_gemm_kernel<kBN, 1, kStages, EPI_RESID>, grid, blk, Small::SMEM, s, 0, *a, *b, *b2,
                                    g, p->err));
@@ -223,9 +212,6 @@ int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g0, cudaStream_t s) {
         return launched(launch_pdl(tc_gemm_kernel<kBN, 1, kStages, EPI_QKV>, grid, blk, Small::SMEM, s, 0, *a, *b, *b2, g,
                                    p->err));
     switch (epi) {
-        case EPI_PARTIAL:
-            return launched(launch_pdl(tc_gemm_kernel<kBN, 2, kStages, EPI_PARTIAL>, grid, blk, Big::SMEM, s, 0, *a, *b,
-                                       *b2, g, p->err));
         case EPI_SWIGLU:
             return launched(launch_pdl(tc_gemm_kernel<kBN, 2, kStages, EPI_SWIGLU>, grid, blk, Big::SMEM, s, 0, *a, *b,
                                        *b2, g, p->err));
@@ -238,8 +224,9 @@ int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g0, cudaStream_t s) {
         case EPI_QKV:
             return launched(launch_pdl(tc_gemm_kernel<kBN, 2, kStages, EPI_QKV>, grid, blk, Big::SMEM, s, 0, *a, *b, *b2,
                                        g, p->err));
+        default:
+            return -1;
     }
-    return -1;
 }
 
 }  // namespace focus

@@ -4,8 +4,6 @@
 
 namespace focus {
 
-enum WeightId { W_QKV = 0, W_O = 1, W_GATEUP = 2, W_DOWN = 3, W_LM = 4 };
-
 struct TcWeights {
     int L;
     const void* const* wqkv;
@@ -24,6 +22,6 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
                    int rows_c, int lm_tiles_cap, int* err);
 void tc_plan_destroy(TcPlan* p);
 int tc_lm_tiles(const TcPlan* p);
-int tc_gemm(TcPlan* p, Epi epi, int wid, const GemmArgs& g, cudaStream_t s);
+int tc_gemm(TcPlan* p, Epi epi, const GemmArgs& g, cudaStream_t s);
 
 }  // namespace focus

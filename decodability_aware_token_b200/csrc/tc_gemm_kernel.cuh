@@ -143,7 +143,6 @@ __device__ __forceinline__ bf16* qkv_dst(const GemmArgs& g, int row, int head, i
 
 __device__ __forceinline__ void named_sync_epilogue() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-constexpr int kMaxReduceSplits = 8;  // split-K slices the fused reduction sums (the launcher never uses more)
 
 template <int BN, int MSUB, int STAGES>
 struct TcShape {
@@ -268,34 +267,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
             const int row = m0 + ms * 128 + quarter * 32 + lane;
             const bool live = ok && row < M && nk > 0;
             const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + ms * BN;
-            if (EPI == EPI_PARTIAL) {
-                float* out = g.part + (size_t)split * g.split_stride + (size_t)row * g.N + (size_t)n_tile * BN;
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    float v[32];
-                    tmem_ld32(tbase + c0, v);
-                    if (live) {
-                        float4* o4 = reinterpret_cast<float4*>(out + c0);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) o4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                    }
-                }
-            } else if (EPI == EPI_RESID || EPI == EPI_QKV) {
-                if (gridDim.z > 1) {
-                    // split K: leave this split's partial tile; the tile's last CTA reduces below
-                    float* out = g.part + (size_t)split * g.split_stride + (size_t)row * g.N + (size_t)n_tile * BN;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < BN; c0 += 32) {
-                        float v[32];
-                        tmem_ld32(tbase + c0, v);
-                        if (live) {
-                            float4* o4 = reinterpret_cast<float4*>(out + c0);
-#pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                o4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                        }
-                    }
-                } else if (EPI == EPI_RESID) {
+            if (EPI == EPI_RESID || EPI == EPI_QKV) {
+                if (EPI == EPI_RESID) {
                     float* xr = g.resid + (size_t)row * g.N + (size_t)n_tile * BN;
 #pragma unroll 1
                     for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -405,83 +378,6 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
                     g.lm_max[idx] = mx;
                     g.lm_sum[idx] = se;
                     g.lm_arg[idx] = arg;
-                }
-            }
-        }
-        if constexpr (EPI == EPI_RESID || EPI == EPI_QKV) {
-            if (gridDim.z > 1) {  // block-uniform: every epilogue thread reaches both barriers
-                // last split CTA of this output tile: sum the splits in order and apply the epilogue
-                // (a split that timed out still counts its arrival; its outputs are flagged invalid)
-                __shared__ int last_split;
-                __threadfence();
-                named_sync_epilogue();
-                const int tile_id = blockIdx.y * gridDim.x + blockIdx.x;
-                if (warp == 2 && lane == 0) last_split = atomicAdd(&g.counters[tile_id], 1) == (int)gridDim.z - 1;
-                named_sync_epilogue();
-                if (last_split) {
-                    __threadfence();
-                    const int ew = warp - 2;
-                    const int col = lane * 4;  // BN == 128: 32 lanes x 4 columns
-                    const int rmax = M < m0 + S::BM ? M : m0 + S::BM;
-                    const int nsp = (int)gridDim.z;
-                    // 4 rows per pass, every split of them loaded before any is summed (one L2 round trip),
-                    // then summed in split order
-                    for (int r0 = m0 + ew; r0 < rmax; r0 += 16) {
-                        float4 pv[4][kMaxReduceSplits];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-#pragma unroll
-                            for (int sp = 0; sp < kMaxReduceSplits; ++sp)
-                                pv[q][sp] = (sp < nsp && r0 + 4 * q < rmax)
-                                                ? __ldcg(reinterpret_cast<const float4*>(
-                                                      g.part + (size_t)sp * g.split_stride +
-                                                      (size_t)(r0 + 4 * q) * g.N + (size_t)n_tile * BN + col))
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int row = r0 + 4 * q;
-                        if (row >= rmax) continue;  // warp-uniform (the row depends on the warp only)
-                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                        for (int sp = 0; sp < kMaxReduceSplits; ++sp) {
-                            acc.x += pv[q][sp].x;
-                            acc.y += pv[q][sp].y;
-                            acc.z += pv[q][sp].z;
-                            acc.w += pv[q][sp].w;
-                        }
-                        if (EPI == EPI_RESID) {
-                            float4* x4 = reinterpret_cast<float4*>(g.resid + (size_t)row * g.N + (size_t)n_tile * BN + col);
-                            float4 x = *x4;
-                            x.x += acc.x;
-                            x.y += acc.y;
-                            x.z += acc.z;
-                            x.w += acc.w;
-                            *x4 = x;
-                        } else {
-                            const int head = n_tile;
-                            int b, j, pos;
-                            qkv_row(g, row, b, j, pos);
-                            float v[4] = {acc.x, acc.y, acc.z, acc.w};
-                            float o4[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float partner = __shfl_xor_sync(0xffffffffu, v[e], 16);  // column +- 64
-                                if (head < g.Hq + g.Hkv) {
-                                    const int i = (col + e) & 63;
-                                    float cn, sn;
-                                    rope_cs(g, pos, i, cn, sn);
-                                    o4[e] = col < 64 ? v[e] * cn - partner * sn : v[e] * cn + partner * sn;
-                                } else {
-                                    o4[e] = v[e];
-                                }
-                            }
-                            bf16* dst = qkv_dst(g, row, head, b, j) + col;
-                            *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(o4[0], o4[1]);
-                            *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __floats2bfloat162_rn(o4[2], o4[3]);
-                        }
-                    }
-                    }
-                    if (warp == 2 && lane == 0) g.counters[tile_id] = 0;  // ready for the next launch
                 }
             }
         }
