@@ -260,6 +260,31 @@ def make_batch(shape: ModelShape, work: Workload, seed: int, device="cpu",
     }
 
 
+def with_block_pages(batch: dict, block: int) -> dict:
+    """A copy of `batch` whose page tables also cover positions P_b .. P_b + block - 1 of every request
+    (the block about to be committed to the prefix): the last prefix page is shared, further pages are
+    appended to the pool (zero-filled) in request order.  Input preparation only: no step arithmetic."""
+    pool, table, plen = batch["kv_pool"], batch["page_table"].cpu(), batch["prefix_len"].cpu()
+    S = int(pool.shape[4])
+    N = int(table.shape[0])
+    need = [(int(p) + block + S - 1) // S for p in plen]
+    have = [(int(p) + S - 1) // S for p in plen]
+    width = max(int(table.shape[1]), max(need))
+    new_table = torch.full((N, width), -1, dtype=torch.int32)
+    new_table[:, : table.shape[1]] = table
+    n_old = int(pool.shape[0])
+    at = n_old
+    for b in range(N):
+        for i in range(have[b], need[b]):
+            new_table[b, i] = at
+            at += 1
+    extra = torch.zeros((at - n_old,) + tuple(pool.shape[1:]), dtype=pool.dtype, device=pool.device)
+    out = dict(batch)
+    out["kv_pool"] = torch.cat([pool, extra], 0)
+    out["page_table"] = new_table.to(batch["page_table"].device)
+    return out
+
+
 def make_case(name: str = "tiny", seed: Optional[int] = None, device="cpu", *, shape: Optional[ModelShape] = None,
               work: Optional[Workload] = None, lm_boost_frac: float = 0.0, lm_boost: float = 50.0,
               **work_overrides) -> Case:

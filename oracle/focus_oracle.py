@@ -430,3 +430,71 @@ def focus_step(shape, model: dict, batch: dict, *, tau: float, k_min: int, k_max
     return OracleResult(importance, delta, keep_count, retained, offsets, row_map, hidden, conf, top_id, decoded,
                         new_tokens, new_mask.astype(np.uint8), ibc, cut_gap, tau_gap, log_conf, margin,
                         thr_gap, fb_gap)
+
+
+# --------------------------------------------------------------------------
+# around the step: one block to completion, then its K/V into the prefix
+# --------------------------------------------------------------------------
+
+def commit_block(kv_pool, ibc, prefix_len, page_table):
+    """Write every request's block K/V into its prefix pages at positions P_b .. P_b + B - 1 and grow the
+    prefix by B.
+
+    Project page, Overview -- Motivation: the prefix is served from an exactly cached KV; a block that
+    has been decoded becomes part of that prefix.  `ibc` is the intra-block cache [N, L, 2, Hkv, B, d]
+    after the block's final refresh; the pages hold [pages, L, 2, Hkv, S, d].  Returns (pool, prefix_len)
+    as new float64 / int64 arrays."""
+    pool = _f64(kv_pool).copy()
+    cache = _f64(ibc)
+    plen = _i64(prefix_len).copy()
+    table = _i64(page_table)
+    S = pool.shape[4]
+    N, B = cache.shape[0], cache.shape[4]
+    for b in range(N):
+        for j in range(B):
+            pos = int(plen[b]) + j
+            page = int(table[b, pos // S])
+            pool[page, :, :, :, pos % S, :] = cache[b, :, :, :, j, :]
+    return pool, plen + B
+
+
+@dataclasses.dataclass
+class BlockResult:
+    steps: list                  # OracleResult of every decoding step (the first one dense)
+    block_tokens: np.ndarray     # [N, B] the decoded block
+    ibc: np.ndarray              # [N, L, 2, Hkv, B, d] after the final dense refresh
+    kv_pool: np.ndarray          # pages after the commit
+    prefix_len: np.ndarray       # [N] grown by B
+
+
+def decode_block(shape, model: dict, batch: dict, *, tau: float, k_min: int, k_max: int, conf_threshold: float,
+                 alpha: float = 1.0, max_steps: Optional[int] = None, storage: str = "f64") -> BlockResult:
+    """Denoise one block to completion and commit it.
+
+    Project page, Overview -- Motivation / Runtime Action: a block is decoded over several denoising
+    steps, each computing the block on top of the cached prefix; FOCUS runs the later layers only on the
+    kept positions, whose fresh K/V refresh the intra-block cache while evicted positions keep theirs.
+    Readings: the block's first step is dense (every position computed, which fills the intra-block
+    cache); then focused steps run until no position is masked (the decode rule's fallback decodes at
+    least one masked position of every request that has one, so at most B steps); the fully decoded
+    block is computed once more densely so that its cache holds the K/V of the final tokens, and that
+    cache is committed to the prefix pages."""
+    B = int(_i64(batch["block_tokens"]).shape[1])
+    max_steps = B if max_steps is None else max_steps
+    state = {k: v for k, v in batch.items()}
+    steps = []
+
+    def run(frac):
+        r = focus_step(shape, model, state, tau=tau, k_min=k_min, k_max=k_max, conf_threshold=conf_threshold,
+                       alpha=alpha, forced_keep_frac=frac, max_keep=B, storage=storage)
+        state["block_tokens"], state["mask"], state["ibc"] = r.block_tokens, r.mask, r.ibc
+        return r
+
+    steps.append(run(1.0))
+    while np.asarray(state["mask"]).any() and len(steps) < max_steps:
+        steps.append(run(-1.0))
+    if np.asarray(state["mask"]).any():
+        raise ValueError("block not decoded within max_steps")
+    refresh = run(1.0)
+    pool, plen = commit_block(state["kv_pool"], refresh.ibc, state["prefix_len"], state["page_table"])
+    return BlockResult(steps, np.asarray(state["block_tokens"]), refresh.ibc, pool, plen)
