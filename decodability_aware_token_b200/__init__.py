@@ -199,6 +199,30 @@ class FocusContext:
                    "focus_step")
         return out
 
+    def commit_block(self, batch: dict, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """Copy the block's K/V (batch["ibc"]) into the prefix pages at positions P_b .. P_b + B - 1 and
+        add B to batch["prefix_len"] (both in place; the page table must map those positions)."""
+        N, B = batch["block_tokens"].shape
+        cb, _, _ = self._marshal(batch, StepParams(), self.alloc_outputs(N, B))
+        with torch.cuda.device(self.device):
+            s = stream if stream is not None else torch.cuda.current_stream(self.device)
+            _check(self._lib.focus_commit_block(self._ctx, C.byref(cb), C.c_void_p(s.cuda_stream)), "focus_commit_block")
+
+    def decode_block(self, batch: dict, params: StepParams, max_steps: Optional[int] = None,
+                     out: Optional[StepOutputs] = None, stream: Optional[torch.cuda.Stream] = None):
+        """Decode the block to completion (dense first step, focused steps, dense refresh) and commit it;
+        returns (outputs of the last call, number of decoding steps).  Synchronises after every step."""
+        N, B = batch["block_tokens"].shape
+        if out is None:
+            out = self.alloc_outputs(N, B)
+        cb, cp, co = self._marshal(batch, params, out)
+        steps = C.c_int32(0)
+        with torch.cuda.device(self.device):
+            s = stream if stream is not None else torch.cuda.current_stream(self.device)
+            _check(self._lib.focus_decode_block(self._ctx, C.byref(cb), C.byref(cp), int(max_steps or B), C.byref(co),
+                                                C.byref(steps), C.c_void_p(s.cuda_stream)), "focus_decode_block")
+        return out, int(steps.value)
+
     def last_step_launches(self) -> int:
         """Kernels the most recent step enqueued."""
         return int(self._lib.focus_last_step_launches(self._ctx))

@@ -16,6 +16,7 @@
 
 #include "launch.h"
 #include "tc_gemm.h"
+#include "block.h"
 
 using namespace focus;
 
@@ -36,6 +37,7 @@ struct focus_ctx {
     int32_t *row_req, *row_pos, *row_src, *n_rows, *lm_arg;
     double* inv_freq;
     float2* rope_tab;     // bf16 path: [rope_positions][head_dim / 2] (cos, sin)
+    int32_t* masked_count;  // block loop: masked positions left after a step
     int* err;
     float *att_part_o, *att_part_ml, *att_sb;
     int* att_counters;
@@ -126,10 +128,11 @@ Layout plan(const focus_model_cfg* c, const focus_limits* l) {
         split * (size_t)kAttnSplitCap * 4,                  // 20 arrival counters
         rows_c * 4, rows_c * 4,                             // 21-22 per-row confidence / top id
         split * rope_positions(l) * (size_t)c->head_dim / 2 * 8,  // 23 RoPE (cos, sin) table
+        64,                                                 // 24 block loop: masked-position count
     };
     Layout lay{};
     size_t at = 0;
-    for (int i = 0; i < 24; ++i) {
+    for (int i = 0; i < 25; ++i) {
         lay.off[i] = at;
         at = align_up(at + sizes[i], 1024);
     }
@@ -425,6 +428,7 @@ int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_l
     c->lm_arg = reinterpret_cast<int32_t*>(base + lay.off[14]);
     c->inv_freq = reinterpret_cast<double*>(base + lay.off[15]);
     c->rope_tab = reinterpret_cast<float2*>(base + lay.off[23]);
+    c->masked_count = reinterpret_cast<int32_t*>(base + lay.off[24]);
     c->err = reinterpret_cast<int*>(base + lay.off[16]);
     c->att_part_o = reinterpret_cast<float*>(base + lay.off[17]);
     c->att_part_ml = reinterpret_cast<float*>(base + lay.off[18]);
@@ -513,6 +517,72 @@ int focus_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (c->cfg.dtype == FOCUS_DTYPE_BF16) return run_step<bf16>(c, in, p, out, s, k_cap);
     return run_step<float>(c, in, p, out, s, k_cap);
+}
+
+int focus_commit_block(focus_ctx* c, const focus_batch* in, void* stream) {
+    if (!c || !in) return FOCUS_ERR_INVALID_ARG;
+    const int N = in->n_requests, B = in->block_size;
+    if (N < 0 || B <= 0 || in->page_size <= 0 || in->n_pages <= 0) return FOCUS_ERR_INVALID_ARG;
+    if (N > c->lim.max_requests || B > c->lim.max_block) return FOCUS_ERR_LIMITS;
+    if (!in->prefix_len || !in->page_table || !in->ibc || !in->kv_pool) return FOCUS_ERR_INVALID_ARG;
+    if (N == 0) return FOCUS_OK;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != c->device) return FOCUS_ERR_INVALID_ARG;
+    CommitArgs a{};
+    a.ibc = in->ibc;
+    // the step only reads the pages and prefix lengths; the commit is the one call that writes them
+    a.kv_pool = const_cast<void*>(in->kv_pool);
+    a.prefix_len = const_cast<int32_t*>(in->prefix_len);
+    a.page_table = in->page_table;
+    a.N = N;
+    a.L = c->dm.L;
+    a.Hkv = c->dm.Hkv;
+    a.B = B;
+    a.d = c->dm.d;
+    a.S = in->page_size;
+    a.max_pages = c->lim.max_pages_per_req;
+    a.n_pages = in->n_pages;
+    a.elt = (int)c->elt;
+    a.err = c->err;
+    return launch_commit_block(a, static_cast<cudaStream_t>(stream)) < 0 ? FOCUS_ERR_CUDA : FOCUS_OK;
+}
+
+int focus_decode_block(focus_ctx* c, const focus_batch* in, const focus_params* p, int32_t max_steps,
+                       focus_step_out* out, int32_t* steps_taken, void* stream) {
+    if (!c || !in || !p || !out || max_steps < 1) return FOCUS_ERR_INVALID_ARG;
+    if (steps_taken) *steps_taken = 0;
+    const int N = in->n_requests, B = in->block_size;
+    if (B > c->lim.max_keep) return FOCUS_ERR_LIMITS;  // the dense steps keep every position
+    if (p->forced_keep_idx) return FOCUS_ERR_INVALID_ARG;
+    if (N <= 0) return N == 0 ? FOCUS_OK : FOCUS_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    focus_params dense = *p, focused = *p;
+    dense.forced_keep_frac = 1.f;
+    focused.forced_keep_frac = -1.f;
+    auto masked_left = [&](int32_t* left) {
+        if (launch_count_masked(in->mask, N * B, c->masked_count, s) < 0 ||
+            cudaMemcpyAsync(left, c->masked_count, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return FOCUS_ERR_CUDA;
+        return FOCUS_OK;
+    };
+    // the block's first step is dense; then focused steps until nothing is masked
+    int rc = focus_step(c, in, &dense, out, stream);
+    int steps = 1;
+    int32_t left = 0;
+    if (rc == FOCUS_OK) rc = masked_left(&left);
+    while (rc == FOCUS_OK && left > 0 && steps < max_steps) {
+        rc = focus_step(c, in, &focused, out, stream);
+        ++steps;
+        if (rc == FOCUS_OK) rc = masked_left(&left);
+    }
+    if (steps_taken) *steps_taken = steps;
+    if (rc != FOCUS_OK) return rc;
+    if (left > 0) return FOCUS_ERR_LIMITS;  // not decoded within max_steps: nothing is committed
+    // one dense refresh of the decoded block (its cache then holds the final tokens' K/V), then commit
+    rc = focus_step(c, in, &dense, out, stream);
+    if (rc != FOCUS_OK) return rc;
+    return focus_commit_block(c, in, stream);
 }
 
 int focus_destroy(focus_ctx* c) {

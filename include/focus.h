@@ -176,6 +176,35 @@ int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_l
  * the same context must not overlap in time (the workspace is shared). */
 int focus_step(focus_ctx* ctx, const focus_batch* in, const focus_params* p, focus_step_out* out, void* stream);
 
+/* ---- around the step: one block to completion --------------------------------
+ * The loop a block-diffusion decoder runs around the focused step (project page, Overview --
+ * Motivation: every denoising step computes the block on top of an exactly cached prefix; a decoded
+ * block becomes part of that prefix).  Readings: the block's first step is dense (forced keep
+ * fraction 1, filling the intra-block cache); focused steps follow until no position is masked (the
+ * decode rule's fallback decodes at least one masked position of every request that has one, so at
+ * most B steps); the decoded block is computed once more densely so that its cache holds the final
+ * tokens' K/V; that cache is committed to the prefix pages.
+ *
+ * focus_commit_block copies in->ibc [N, L, 2, Hkv, B, d] into in->kv_pool at positions
+ * P_b .. P_b + B - 1 of every request (pages from in->page_table, which must already map those
+ * positions; the last prefix page may be shared) and then adds B to in->prefix_len[b].  It is the one
+ * call that WRITES kv_pool and prefix_len (the pointers are declared const for the step, which only
+ * reads them).  Asynchronous, two kernel launches.  Positions without a valid page set
+ * FOCUS_DEVERR_PAGE_ID and are skipped; a prefix length outside [0, max_pages_per_req * page_size] sets
+ * FOCUS_DEVERR_PREFIX and leaves that request untouched.  Returns FOCUS_OK, FOCUS_ERR_INVALID_ARG,
+ * FOCUS_ERR_LIMITS or FOCUS_ERR_CUDA. */
+int focus_commit_block(focus_ctx* ctx, const focus_batch* in, void* stream);
+
+/* Run the loop above on `in` with `p` (p->forced_keep_frac is ignored: the loop's own steps are dense
+ * or adaptive; p->forced_keep_idx must be NULL) and commit the block.  `out` receives each step's
+ * outputs in turn (the last one is the dense refresh, which decodes nothing).  Synchronises `stream`
+ * after every step to read how many positions are still masked, so it cannot be captured in a CUDA
+ * graph.  Needs limits.max_keep >= B.  *steps_taken (if not NULL) receives the number of decoding
+ * steps.  If positions are still masked after max_steps decoding steps, nothing is committed and
+ * FOCUS_ERR_LIMITS is returned.  Other returns as for focus_step / focus_commit_block. */
+int focus_decode_block(focus_ctx* ctx, const focus_batch* in, const focus_params* p, int32_t max_steps,
+                       focus_step_out* out, int32_t* steps_taken, void* stream);
+
 /* Free the workspace.  Synchronises the device first.  NULL is accepted. */
 int focus_destroy(focus_ctx* ctx);
 
