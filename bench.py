@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--eager", action="store_true", help="time eager focus_step calls instead of graph replays")
     ap.add_argument("--layers", type=int, default=None, help="override the layer count (profiling cases)")
     ap.add_argument("--requests", type=int, default=None, help="override the request count (profiling cases)")
+    ap.add_argument("--mode", choices=["step", "block"], default="step",
+                    help="step: one focused step (the default measurement); block: whole blocks decoded to "
+                         "completion and committed (dense first step, focused steps, dense refresh, commit)")
     return ap.parse_args()
 
 
@@ -272,6 +275,63 @@ def whole_job_rate(total_units: float, max_ms: float) -> float:
     return total_units / (max_ms / 1e3) if max_ms > 0 else 0.0
 
 
+# ------------------------------------------------------------------ whole blocks
+def run_block_mode(args, case, dev, world, barrier):
+    """Decode whole blocks through focus_decode_block: the dense first step, focused steps until nothing is
+    masked (the loop reads the remaining count after every step), the dense refresh and the commit of
+    the block's K/V into the prefix pages.  Each timed block starts from the workload's initial block
+    state and prefix lengths.  tokens/s = masked positions decoded / device time of the blocks."""
+    from decodability_aware_token_b200 import FocusContext, StepParams
+    w, shp = case.work, case.shape
+    N, B = w.n_requests, w.block
+    batch = fs.with_block_pages(case.batch, B)
+    params = StepParams(w.tau, w.k_min, w.k_max, w.conf_threshold, w.alpha, -1.0)
+    ctx = FocusContext(shp, case.model, max_requests=N, max_block=B, max_keep=B,
+                       max_pages_per_req=int(batch["page_table"].shape[1]))
+    init = {k: batch[k].clone() for k in ("block_tokens", "mask", "ibc", "prefix_len")}
+    st = dict(batch)
+    masked = int(init["mask"].sum())
+
+    def one_block():
+        for k, v in init.items():
+            st[k].copy_(v)
+        return ctx.decode_block(st, params)[1]
+
+    for _ in range(max(1, args.warmup)):
+        one_block()
+    torch.cuda.synchronize(dev)
+    K = max(1, min(args.steps, 20))
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tw0 = time.time()
+    ev0.record(stream)
+    steps = [one_block() for _ in range(K)]
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    tw1 = time.time()
+    barrier()
+    sampler.stop()
+    elapsed = ev0.elapsed_time(ev1)
+    max_ms, total = reduce_over_ranks(elapsed, masked * K, world, dev)
+    if int(os.environ.get("RANK", "0")) == 0:
+        line = {
+            "metric": "decoded tokens/s, whole blocks (dense first step, focused steps, dense refresh, commit)",
+            "value": whole_job_rate(total, max_ms), "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_block": max_ms / K, "focused_steps_per_block": statistics.mean(steps) - 1,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": shp.dtype,
+            "data": "synthetic", "clocks": sampler.summary(tw0, tw1),
+            "config": {"workload": args.workload, "mode": "block", "desc": workload_desc(case),
+                       "masked_per_block": masked, "requests_per_gpu": N,
+                       "launch": "eager calls; the loop synchronises after every step to read the masked count"},
+        }
+        print(json.dumps(line), flush=True)
+    ctx.close()
+
+
 # ------------------------------------------------------------------ the GPU arm
 def main():
     args = parse()
@@ -298,6 +358,11 @@ def main():
     case = make_workload(args, rank_seed(base, rank), dev)    # this rank's requests
     w, shp = case.work, case.shape
     N, B = w.n_requests, w.block
+    if args.mode == "block":
+        run_block_mode(args, case, dev, world, barrier)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     params = StepParams(w.tau, w.k_min, w.k_max, w.conf_threshold, w.alpha, w.forced_keep_frac)
     mk = B if w.forced_keep_frac >= 0 else w.k_max
     ctx = FocusContext(shp, case.model, max_requests=N, max_block=B, max_keep=mk,
