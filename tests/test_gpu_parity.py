@@ -272,3 +272,23 @@ def test_kernel_sweep_points_sampled(n, block, frac):
     rep = _sampled_check(case, [0, n - 1])
     del case
     print(rep)
+
+
+# ---------------------------------------------------------------- budget / decode variants
+@pytest.mark.parametrize("alpha", [1.2, 1.5, 1.8])
+@pytest.mark.parametrize("threshold", [0.7, 0.8, 0.9])
+def test_quality_table_knobs(alpha, threshold):
+    """The knobs of the project page's Quality table: the budget multiplier alpha (1.2 / 1.5 / 1.8) and the
+    confidence threshold "Conf." (0.7 / 0.8 / 0.9), with boosted LM-head rows so that the threshold
+    decides (bf16 shape, several tiles)."""
+    case = _case("small_bf16", lm_boost_frac=0.001, lm_boost=25.0)
+    p = step_params(case.work, alpha=alpha, conf_threshold=threshold)
+    gpu = run_gpu(case, p)
+    check(case, p, gpu=gpu)
+
+
+@pytest.mark.parametrize("block", [16, 64])
+def test_other_block_sizes(block):
+    """Block sizes 16 and 64 on the reduced bf16 shape (the project page's efficiency figures use several)."""
+    case = _case("small_bf16", block=block, k_max=min(8, block))
+    check(case, step_params(case.work), _model("small_bf16_b%d" % block, case))
