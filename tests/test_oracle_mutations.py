@@ -108,7 +108,55 @@ def _decode_not_strict(kept, masked, conf, top_id, threshold):
     return {int(kept[t]): int(top_id[t]) for t in dec}, math.inf, math.inf
 
 
-_orig = {n: getattr(fo, n) for n in ("select_positions", "lm_head_conf")}
+def _select_variant(*, count_all=False, floor_budget=False, no_kmin=False, unmasked_first=False):
+    def sel(delta, masked, *, tau, k_min, k_max, alpha=1.0, forced_keep_frac=-1.0):
+        masked = np.asarray(masked).astype(bool)
+        B = len(delta)
+        tau32 = float(np.float32(tau))
+        if forced_keep_frac >= 0:
+            k = min(B, fo._ceil_f32(forced_keep_frac, B))
+            first = (lambda j: 1 if masked[j] else 0) if unmasked_first else (lambda j: 0 if masked[j] else 1)
+            order = sorted(range(B), key=lambda j: (first(j), -delta[j], j))    # slip (optional): key order
+            return sorted(order[:k]), math.inf, math.inf
+        eligible = [j for j in range(B) if masked[j]]
+        pool = range(B) if count_all else eligible                                # slip (optional): count all
+        c = sum(1 for j in pool if delta[j] > tau32)
+        k = int(np.floor(np.float32(alpha) * np.float32(c))) if floor_budget else fo._ceil_f32(alpha, c)
+        k = min(k if no_kmin else max(k, k_min), k_max)                           # slip (optional): no k_min
+        k = min(k, len(eligible))
+        order = sorted(eligible, key=lambda j: (-delta[j], j))
+        return sorted(order[:k]), math.inf, math.inf
+    return sel
+
+
+def _importance_block_normalised(p, prefix_len):
+    blk = p[:, :, prefix_len:]
+    return (blk / blk.sum(axis=2, keepdims=True)).sum(axis=(0, 1))               # slip: softmax over block only
+
+
+def _compact_descending(kept, max_keep):
+    return _orig["compact_rows"]([sorted(s, reverse=True) for s in kept], max_keep)  # slip: order reversed
+
+
+def _decode_fallback_any(kept, masked, conf, top_id, threshold):
+    thr = float(np.float32(threshold))
+    cand = [t for t, j in enumerate(kept) if masked[j]]
+    dec = [t for t in cand if conf[t] > thr]
+    if not dec and cand:
+        dec = [max(range(len(kept)), key=lambda t: (conf[t], -kept[t]))]           # slip: fallback may pick unmasked
+    return {int(kept[t]): int(top_id[t]) for t in dec}, math.inf, math.inf
+
+
+def _decode_fallback_high_j(kept, masked, conf, top_id, threshold):
+    thr = float(np.float32(threshold))
+    cand = [t for t, j in enumerate(kept) if masked[j]]
+    dec = [t for t in cand if conf[t] > thr]
+    if not dec and cand:
+        dec = [max(cand, key=lambda t: (conf[t], kept[t]))]                      # slip: higher j wins ties
+    return {int(kept[t]): int(top_id[t]) for t in dec}, math.inf, math.inf
+
+
+_orig = {n: getattr(fo, n) for n in ("select_positions", "lm_head_conf", "compact_rows")}
 
 MUTATIONS = {
     "rope_sign": ("rope", _rope_sign),
@@ -122,6 +170,14 @@ MUTATIONS = {
     "mlp_residual_dropped": ("layer_forward", _layer_variant(mlp_residual=False)),
     "argmax_highest_id": ("lm_head_conf", _lm_head_highest_id),
     "decode_threshold_not_strict": ("threshold_decode", _decode_not_strict),
+    "budget_counts_unmasked_positions": ("select_positions", _select_variant(count_all=True)),
+    "budget_floor_instead_of_ceil": ("select_positions", _select_variant(floor_budget=True)),
+    "budget_without_k_min": ("select_positions", _select_variant(no_kmin=True)),
+    "forced_keep_unmasked_first": ("select_positions", _select_variant(unmasked_first=True)),
+    "importance_softmax_over_block_only": ("importance_from_probs", _importance_block_normalised),
+    "compaction_descending": ("compact_rows", _compact_descending),
+    "fallback_may_pick_unmasked": ("threshold_decode", _decode_fallback_any),
+    "fallback_higher_position_on_ties": ("threshold_decode", _decode_fallback_high_j),
 }
 
 PINS = [getattr(pins, n) for n in sorted(dir(pins)) if n.startswith("test_") and n not in (
