@@ -5,8 +5,9 @@
 //   EPI_RESID:   resid += A B^T (float32 residual stream)
 //   EPI_QKV:     rotary embedding of the query / key heads, queries to q, keys and values to the cache
 //
-// GEMMs of at most 256 rows with the RESID, QKV or SWIGLU epilogue run on the swapped kernel
-// (features on the MMA's M side, tokens on N); the rest on the row-major kernel below.
+// GEMMs of at most 256 rows (the kept rows and the LM head) run on the swapped kernel (features on the
+// MMA's M side, tokens on N, split K over a thread-block cluster); the full-block GEMMs of layers 0-1 on
+// the row-major kernel.
 //
 // One CTA computes a (128 * MSUB) x BN tile (MSUB accumulators of 128 x BN fp32 in TMEM) over a range of
 // 64-wide K blocks.  Warp roles: warp 0 lane 0 issues TMA loads into a STAGES-deep shared-memory ring,
