@@ -41,6 +41,7 @@ constexpr int kStages = 3;      // chunks in the ring (2 in flight while one is 
 constexpr int kHalf = kChunk * 128;         // one [64 keys][64 d] bf16 half-tile: 8 KB
 constexpr int kStageBytes = 4 * kHalf;      // K lo, K hi, V lo, V hi: 32 KB
 constexpr int kPtCache = 512;               // page-table entries cached in shared memory
+constexpr int kAttnSmem = kStages * kStageBytes + 1024;  // dynamic shared memory: 97 KB, two CTAs per SM
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -537,7 +538,13 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_const
 }  // namespace
 
 bool configure_attention_tc_kernels() {
-    return max_shared_carveout((const void*)attention_tc_kernel<true>) &&
+    // once per context (device current): the shared-memory opt-in is not a stream operation, so it is
+    // never made at launch time, where it would break stream capture
+    return cudaFuncSetAttribute(attention_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) ==
+               cudaSuccess &&
+           cudaFuncSetAttribute(attention_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) ==
+               cudaSuccess &&
+           max_shared_carveout((const void*)attention_tc_kernel<true>) &&
            max_shared_carveout((const void*)attention_tc_kernel<false>);
 }
 
@@ -572,19 +579,7 @@ int launch_attention_tc(const AttnArgs& a, int q_tiles, cudaStream_t s) {
     } else {
         pool_map = ibc_map;  // never used: with no pages every prefix key is invalid
     }
-    const int smem = kStages * kStageBytes + 1024;  // 97 KB: two CTAs per SM
-    // the shared-memory opt-in is set once per device (not per launch, so launches stay capturable)
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(attention_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(attention_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-                cudaSuccess)
-            return -1;
-        attr_set[dev] = true;
-    }
+    const int smem = kAttnSmem;  // opted in by configure_attention_tc_kernels (at focus_init, per device)
     dim3 grid(a.N, a.Hkv * a.pieces, q_tiles);
     if (a.row_offsets == nullptr)
         return launched(launch_pdl(attention_tc_kernel<true>, grid, dim3(128), smem, s, 0, pool_map, ibc_map, a, q_tiles));
