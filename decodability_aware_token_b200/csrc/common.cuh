@@ -21,12 +21,15 @@ template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __flo
 __device__ __forceinline__ void raise_err(int* err, int bit) { atomicOr(err, bit); }
 
 // Programmatic dependent launch: every kernel of the step is launched so that it may start while its
-// predecessor drains.  On entry it lets its own successor launch, then waits until the predecessor has
-// completed and its memory is visible; nothing is read or written before that wait.  (Without a
-// programmatic launch both are no-ops.)
+// predecessor drains.  On entry it lets its own successor launch (pdl_trigger), then waits until the
+// predecessor has completed and its memory is visible (pdl_wait).  Before that wait a kernel touches
+// nothing that an earlier kernel of the step writes: only the model weights, which no kernel writes, may
+// be read there.  (Without a programmatic launch both are no-ops.)
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_entry() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_trigger();
+    pdl_wait();
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

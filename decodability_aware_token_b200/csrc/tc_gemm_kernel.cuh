@@ -25,6 +25,15 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
+// Raise the bytes the current phase waits for without arriving (the arrival comes later).
+__device__ __forceinline__ void mbar_add_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -162,7 +171,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
                                                          const __grid_constant__ CUtensorMap tmB,
                                                          const __grid_constant__ CUtensorMap tmB2, GemmArgs g,
                                                          int* err) {
-    pdl_entry();
+    pdl_trigger();
     using S = TcShape<BN, MSUB, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -170,9 +179,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
     __shared__ __align__(8) uint64_t accum_bar;
     __shared__ uint32_t tmem_slot;
 
-    const int M = g.M_dev ? *g.M_dev : g.M_bound;
     const int m0 = blockIdx.y * S::BM;
-    if (m0 >= M) return;  // whole CTA, before any barrier or TMEM use
+    if (m0 >= g.M_bound) return;  // whole CTA, before any barrier, copy or TMEM use
     const int n_tile = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -183,6 +191,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
     const int kb0 = (int)((long long)nk_all * split / splits);
     const int kb1 = (int)((long long)nk_all * (split + 1) / splits);
     const int nk = kb1 - kb0;
+    const int n_pre = min(nk, STAGES);  // stages whose weight tiles go out before the programmatic wait
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -202,29 +211,59 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
+    // the weight (B) tiles of the first stages depend on nothing an earlier kernel writes
+    auto load_b = [&](int s, int kx) {
+        uint8_t* b_dst = smem + s * S::STAGE_BYTES + S::A_BYTES;
+        if (EPI == EPI_SWIGLU) {
+            tma_load_2d(&tmB, &full_bar[s], b_dst, kx, n_tile * (BN / 2));
+            tma_load_2d(&tmB2, &full_bar[s], b_dst + (BN / 2) * BK * 2, kx, n_tile * (BN / 2));
+        } else {
+            tma_load_2d(&tmB, &full_bar[s], b_dst, kx, n_tile * BN);
+        }
+    };
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
+        if (EPI == EPI_SWIGLU) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB2) : "memory");
+        for (int s = 0; s < n_pre; ++s) {  // fresh stages: nothing to wait for
+            mbar_add_tx(&full_bar[s], (uint32_t)S::B_BYTES);
+            load_b(s, (kb0 + s) * BK);
+        }
+    }
+    pdl_wait();
+
+    const int M = g.M_dev ? *g.M_dev : g.M_bound;
+    if (m0 >= M) {  // whole CTA: let the early weight copies land, release TMEM, leave
+        if (warp == 0 && lane == 0)
+            for (int s = 0; s < n_pre; ++s) {
+                mbar_arrive(&full_bar[s]);
+                mbar_wait(&full_bar[s], 0u, err);
+            }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (warp == 1)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)S::TMEM_COLS)
+                         : "memory");
+        return;
+    }
 
     if (warp == 0) {
         if (lane == 0) {
             // ---- TMA producer
-            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
-            if (EPI == EPI_SWIGLU) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB2) : "memory");
             int issued = 0;
             for (int i = 0; i < nk; ++i) {
                 const int s = i % STAGES;
                 const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-                if (!mbar_wait(&empty_bar[s], ph ^ 1u, err)) break;
-                uint8_t* a_dst = smem + s * S::STAGE_BYTES;
-                uint8_t* b_dst = a_dst + S::A_BYTES;
-                mbar_expect_tx(&full_bar[s], S::STAGE_BYTES);
                 const int kx = (kb0 + i) * BK;
-                tma_load_2d(&tmA, &full_bar[s], a_dst, kx, m0);
-                if (EPI == EPI_SWIGLU) {
-                    tma_load_2d(&tmB, &full_bar[s], b_dst, kx, n_tile * (BN / 2));
-                    tma_load_2d(&tmB2, &full_bar[s], b_dst + (BN / 2) * BK * 2, kx, n_tile * (BN / 2));
+                if (i < n_pre) {  // weight tile already on its way: arrive with the activation bytes
+                    mbar_expect_tx(&full_bar[s], S::A_BYTES);
                 } else {
-                    tma_load_2d(&tmB, &full_bar[s], b_dst, kx, n_tile * BN);
+                    if (!mbar_wait(&empty_bar[s], ph ^ 1u, err)) break;
+                    mbar_expect_tx(&full_bar[s], S::STAGE_BYTES);
+                    load_b(s, kx);
                 }
+                tma_load_2d(&tmA, &full_bar[s], smem + s * S::STAGE_BYTES, kx, m0);
                 ++issued;
             }
             // never leave with copies in flight: wait (bounded) for the last stages issued
@@ -445,20 +484,21 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap tmW2,
                                                           const __grid_constant__ CUtensorMap tmX, GemmArgs g,
                                                           int* err) {
-    pdl_entry();
+    pdl_trigger();
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[kTMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kTMaxStages];
     __shared__ __align__(8) uint64_t accum_bar;
     __shared__ uint32_t tmem_slot;
 
-    const int M = min(g.M_dev ? *g.M_dev : g.M_bound, kTMaxTok);  // the launcher keeps M_bound <= 256
-    if (M <= 0) return;  // the whole grid, before any barrier or TMEM use
-    const int x_boxes = (M + 31) / 32;
-    const int n_cols = x_boxes * 32;               // MMA N and TMEM columns read back
-    const uint32_t tmem_cols = n_cols <= 32 ? 32u : n_cols <= 64 ? 64u : n_cols <= 128 ? 128u : 256u;
-    const int stage_bytes = kTW + x_boxes * kTXBox;  // a multiple of 1024 (swizzle atom alignment)
-    const int nst = min(kTMaxStages, kTRing / stage_bytes);
+    // Before the programmatic-launch wait only what the launch fixes is known: the token bound, the K
+    // slice and the weights.  The ring keeps its weight tiles apart from its token tiles (weights of
+    // stage s at s x 16 KB, token tiles after the last weight stage), so the first stages' weight tiles
+    // can be fetched while the predecessor drains; the live token count, read after the wait, only
+    // sets where the token tiles go and how many stages the ring holds.
+    const int Mb = min(g.M_bound, kTMaxTok);  // the launcher keeps M_bound in [1, 256]
+    const int xb_bound = (Mb + 31) / 32;
+    const uint32_t tmem_cols = xb_bound <= 1 ? 32u : xb_bound <= 2 ? 64u : xb_bound <= 4 ? 128u : 256u;
     const int n_tile = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -469,9 +509,11 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
     const int nk = (int)((long long)nk_all * (split + 1) / splits) - kb0;
     // output features of the tile: 128 (QKV: one head; residual GEMMs; LM head), or 64 gate + 64 up (SwiGLU)
     const int fbase = EPI == EPI_SWIGLU ? n_tile * 64 : n_tile * 128;
+    // stages whose weight tiles go out before the wait: as many as the ring holds at the token bound
+    const int n_pre = min(nk, min(kTMaxStages, kTRing / (kTW + xb_bound * kTXBox)));
 
     if (threadIdx.x == 0) {
-        for (int st = 0; st < nst; ++st) {
+        for (int st = 0; st < kTMaxStages; ++st) {
             mbar_init(&full_bar[st], 1);
             mbar_init(&empty_bar[st], 1);
         }
@@ -488,26 +530,58 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmX) : "memory");
+        if (EPI == EPI_SWIGLU) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW2) : "memory");
+        for (int st = 0; st < n_pre; ++st) {  // fresh stages: nothing to wait for
+            mbar_add_tx(&full_bar[st], (uint32_t)kTW);
+            uint8_t* w_dst = smem + st * kTW;
+            tma_load_2d(&tmW, &full_bar[st], w_dst, (kb0 + st) * BK, fbase);
+            if (EPI == EPI_SWIGLU) tma_load_2d(&tmW2, &full_bar[st], w_dst + kTW / 2, (kb0 + st) * BK, fbase);
+        }
+    }
+    pdl_wait();
+
+    const int M = min(g.M_dev ? *g.M_dev : Mb, Mb);
+    if (M <= 0) {  // the whole grid: let the early weight copies land, release TMEM, leave
+        if (warp == 0 && lane == 0)
+            for (int st = 0; st < n_pre; ++st) {
+                mbar_arrive(&full_bar[st]);
+                mbar_wait(&full_bar[st], 0u, err);
+            }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (warp == 1)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols) : "memory");
+        return;
+    }
+    const int x_boxes = (M + 31) / 32;
+    const int n_cols = x_boxes * 32;               // MMA N and TMEM columns read back (<= tmem_cols)
+    const int x_stage = x_boxes * kTXBox;          // token-tile bytes of a stage (a multiple of 1024)
+    const int nst = min(kTMaxStages, kTRing / (kTW + x_stage));  // >= n_pre, since M <= Mb
+    uint8_t* xring = smem + nst * kTW;             // 1024-aligned (swizzle atom)
     float* park = reinterpret_cast<float*>(smem);  // [token][kTPark] features, once the ring is idle
 
     if (warp == 0) {
         if (lane == 0) {
             // ---- TMA producer
-            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmX) : "memory");
-            if (EPI == EPI_SWIGLU) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmW2) : "memory");
-            const uint32_t bytes = (uint32_t)stage_bytes;
             int issued = 0;
             for (int i = 0; i < nk; ++i) {
                 const int st = i % nst;
                 const uint32_t ph = (uint32_t)(i / nst) & 1u;
-                if (!mbar_wait(&empty_bar[st], ph ^ 1u, err)) break;
-                uint8_t* w_dst = smem + st * stage_bytes;
-                uint8_t* x_dst = w_dst + kTW;
-                mbar_expect_tx(&full_bar[st], bytes);
+                uint8_t* w_dst = smem + st * kTW;
+                uint8_t* x_dst = xring + st * x_stage;
                 const int kx = (kb0 + i) * BK;
-                tma_load_2d(&tmW, &full_bar[st], w_dst, kx, fbase);
-                if (EPI == EPI_SWIGLU) tma_load_2d(&tmW2, &full_bar[st], w_dst + kTW / 2, kx, fbase);
+                if (i < n_pre) {  // weight tile already on its way: arrive with the token bytes
+                    mbar_expect_tx(&full_bar[st], (uint32_t)x_stage);
+                } else {
+                    if (!mbar_wait(&empty_bar[st], ph ^ 1u, err)) break;
+                    mbar_expect_tx(&full_bar[st], (uint32_t)(kTW + x_stage));
+                    tma_load_2d(&tmW, &full_bar[st], w_dst, kx, fbase);
+                    if (EPI == EPI_SWIGLU) tma_load_2d(&tmW2, &full_bar[st], w_dst + kTW / 2, kx, fbase);
+                }
                 for (int bx = 0; bx < x_boxes; ++bx)
                     tma_load_2d(&tmX, &full_bar[st], x_dst + bx * kTXBox, kx, bx * 32);
                 ++issued;
@@ -526,8 +600,8 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
                 const uint32_t ph = (uint32_t)(i / nst) & 1u;
                 if (!mbar_wait(&full_bar[st], ph, err)) break;
                 tc_fence_after();
-                const uint32_t w_addr = smem_u32(smem + st * stage_bytes);
-                const uint32_t x_addr = w_addr + kTW;
+                const uint32_t w_addr = smem_u32(smem + st * kTW);
+                const uint32_t x_addr = smem_u32(xring + st * x_stage);
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
                     mma_bf16(tmem, smem_desc_sw128(w_addr + kk * 32), smem_desc_sw128(x_addr + kk * 32), idesc,
