@@ -7,9 +7,10 @@
 //
 // Work unit (one CTA): request b, KV head g, and a tile of up to 64 query vectors of that group
 // (query vector qi = row * G + head-in-group).  Keys are walked in 64-key chunks: the prefix in page
-// order (page-table lookups per 16-byte copy, so any page size works), then the block's B keys from the
-// intra-block cache as the last chunk.  Chunks are double-buffered through XOR-swizzled shared memory
-// with cp.async.  The 4 warps split the work as RT row tiles x KS key slices (RT * KS = 4): 64 query
+// order (each page's K and V rows copied by TMA with the 128-byte swizzle; pages of 16, 32 or 64
+// tokens), then the block's B keys from the intra-block cache as the last chunk.  A ring of three chunk
+// stages keeps two chunks in flight while one is consumed; the first prefix chunks are requested before
+// the programmatic-launch wait.  The 4 warps split the work as RT row tiles x KS key slices (RT * KS = 4): 64 query
 // vectors -> 4 x 1, 32 -> 2 x 2, <= 16 (the usual ragged case) -> 1 x 4.  Each warp keeps an online
 // softmax (base 2) over its key slice; slices are merged through shared memory at the end.
 //
@@ -134,7 +135,7 @@ template <bool FULL>
 __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_constant__ CUtensorMap pool_map,
                                                               const __grid_constant__ CUtensorMap ibc_map, AttnArgs a,
                                                               int q_tiles) {
-    pdl_entry();
+    pdl_trigger();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* kv = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(8) uint64_t full_bar[kStages];
@@ -147,26 +148,16 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_const
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.Hq / a.Hkv;
-    Unit u;
+    Unit u{};
     u.b = blockIdx.x;
     u.g = blockIdx.y % a.Hkv;
     u.qt = blockIdx.z;
+    // Before the programmatic-launch wait this kernel reads only what no kernel of the step writes: the
+    // prefix lengths, the page table and the prefix pages of the KV pool (the step's first kernel lets
+    // its successors start only after everything queued before the step has completed).  The block's
+    // cache rows, the queries and the kept-row offsets are written earlier in the step and wait.
     u.P = checked_prefix(a.prefix_len, u.b, a.max_pages * a.page_size, a.err);
-    if (FULL) {
-        u.row_base = u.b * a.B;
-        u.n_rows = a.B;
-    } else {
-        u.row_base = a.row_offsets[u.b];
-        u.n_rows = a.row_offsets[u.b + 1] - u.row_base;
-    }
     u.q0 = u.qt * kQTile;
-    u.nq = min(kQTile, u.n_rows * G - u.q0);
-    if (u.nq <= 0) return;
-    const int RT = u.nq <= 16 ? 1 : (u.nq <= 32 ? 2 : 4);
-    const int KS = 4 / RT;
-    const int rt = warp % RT, ks = warp / RT;
-    const int keys_per_warp = kChunk / KS;  // 64, 32 or 16
-    const int key0 = ks * keys_per_warp;
     const int n_prefix_chunks = (u.P + kChunk - 1) / kChunk;
     const int n_chunks = n_prefix_chunks + 1;
     // split-KV: this CTA walks chunks [c_begin, c_end) of the unit's n_chunks
@@ -190,13 +181,36 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_const
     }
     __syncthreads();
     int issued = 0;  // chunks whose copies thread 0 has issued
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages - 1 && c_begin + i < c_end; ++i) {
-            valid_s[i] = issue_chunk(a, u, &pool_map, &ibc_map, kv + i * kStageBytes, &full_bar[i], c_begin + i,
-                                     n_prefix_chunks, pt);
-            ++issued;
-        }
+    // the first query tile of every unit (the only one in the ragged layers' usual case) starts its
+    // leading prefix chunks now
+    if (threadIdx.x == 0 && u.qt == 0)
+        for (; issued < kStages - 1 && c_begin + issued < c_end && c_begin + issued < n_prefix_chunks; ++issued)
+            valid_s[issued] = issue_chunk(a, u, &pool_map, &ibc_map, kv + issued * kStageBytes, &full_bar[issued],
+                                          c_begin + issued, n_prefix_chunks, pt);
+    pdl_wait();
+
+    if (FULL) {
+        u.row_base = u.b * a.B;
+        u.n_rows = a.B;
+    } else {
+        u.row_base = a.row_offsets[u.b];
+        u.n_rows = a.row_offsets[u.b + 1] - u.row_base;
     }
+    u.nq = min(kQTile, u.n_rows * G - u.q0);
+    if (u.nq <= 0) {  // CTA-uniform: let the early copies land, then leave
+        if (threadIdx.x == 0)
+            for (int i = 0; i < issued; ++i) mbar_wait(&full_bar[i], 0u, a.err);
+        return;
+    }
+    const int RT = u.nq <= 16 ? 1 : (u.nq <= 32 ? 2 : 4);
+    const int KS = 4 / RT;
+    const int rt = warp % RT, ks = warp / RT;
+    const int keys_per_warp = kChunk / KS;  // 64, 32 or 16
+    const int key0 = ks * keys_per_warp;
+    if (threadIdx.x == 0)
+        for (; issued < kStages - 1 && c_begin + issued < c_end; ++issued)
+            valid_s[issued] = issue_chunk(a, u, &pool_map, &ibc_map, kv + issued * kStageBytes, &full_bar[issued],
+                                          c_begin + issued, n_prefix_chunks, pt);
 
     // ---- Q fragments (A operand) of this warp's 16 query vectors, straight from global memory
     const int gq = lane >> 2, tq = lane & 3;

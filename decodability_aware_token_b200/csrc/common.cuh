@@ -23,8 +23,10 @@ __device__ __forceinline__ void raise_err(int* err, int bit) { atomicOr(err, bit
 // Programmatic dependent launch: every kernel of the step is launched so that it may start while its
 // predecessor drains.  On entry it lets its own successor launch (pdl_trigger), then waits until the
 // predecessor has completed and its memory is visible (pdl_wait).  Before that wait a kernel touches
-// nothing that an earlier kernel of the step writes: only the model weights, which no kernel writes, may
-// be read there.  (Without a programmatic launch both are no-ops.)
+// nothing that an earlier kernel of the step writes: only inputs that no kernel of the step writes (the
+// model weights; the prefix lengths, page table and prefix pages of the KV pool) may be read there.  The
+// step's first kernel triggers only after its own wait, so nothing queued before the step is still
+// running when any later kernel of the step starts.  (Without a programmatic launch both are no-ops.)
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_entry() {

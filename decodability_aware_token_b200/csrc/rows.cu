@@ -18,7 +18,11 @@ __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(const int32_t*
                                                                   const T* __restrict__ embed,
                                                                   const T* __restrict__ gamma, float eps, int D,
                                                                   float* __restrict__ x, T* __restrict__ h, int* err) {
-    pdl_entry();
+    // the step's first kernel: its successors may start only once everything queued before the step
+    // (a block commit writing the KV pool and prefix lengths, the caller's copies) has completed, so the
+    // step's kernels can read such inputs before their own programmatic-launch wait
+    pdl_wait();
+    pdl_trigger();
     __shared__ float red[32];
     const int r = blockIdx.x, tid = threadIdx.x;
     int tok = tokens[r];
