@@ -14,6 +14,8 @@
 // warp 1 owns the TMEM allocation and its lane 0 issues tcgen05.mma (one elected thread), warps 2..5
 // read the accumulators back with tcgen05.ld (each warp reads its own 32-lane quarter) and run the
 // epilogue.  Operand tiles are K-major with the 128-byte swizzle that TMA writes; no cluster multicast.
+// The weights are written by no kernel of the step, so the producer issues the weight tiles of the first
+// ring stages before the programmatic-launch wait; the activation / token tiles are issued after it.
 // Every mbarrier wait is bounded: on expiry the kernel flags FOCUS_DEVERR_TIMEOUT, still waits (bounded)
 // for its own in-flight copies, frees its TMEM and returns.
 #include <unordered_map>
@@ -29,11 +31,12 @@ using namespace tc;
 
 // ------------------------------------------------------------------ host side
 // Many rows (layers 0-1: N*B rows): 256 x 128 tiles, two 128-row TMEM accumulators sharing each weight
-// tile.  Few rows (layers 2..L-1 and the LM head: at most N*k_max kept rows, typically a few dozen):
-// the swapped kernel for QKV / O / gate-up / down, and 128-row tiles for the LM head, whose CTAs with
-// all rows beyond the live row count exit at once.
+// tile, or 128 x 128 tiles for the residual and QKV GEMMs when 256-row tiles would leave SMs idle.  At
+// most 256 rows (layers 2..L-1 and the LM head: at most N*k_max kept rows, typically a few dozen): the
+// swapped kernel.  More kept rows than that (large batches) take the row-major kernel, whose CTAs with
+// all rows beyond the live row count exit after the wait.
 constexpr int kBN = 128, kStages = 4;
-constexpr int kSmallRows = 256;  // GEMMs with at most this many rows use the few-rows tiles
+constexpr int kSmallRows = 256;  // GEMMs with at most this many rows run on the swapped kernel
 using Big = TcShape<kBN, 2, kStages>;
 using Small = TcShape<kBN, 1, kStages>;
 
