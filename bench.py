@@ -144,16 +144,19 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ roofline bookkeeping
 def algorithmic_work(kclass: str, case: fs.Case, R: int, kept_per_req, plen, splits=1):
-    """(bytes, flops) one launch of `kclass` must move / compute at the minimum (bf16 operands)."""
+    """(bytes, flops) one launch of `kclass` must move / compute at the minimum (operands at the path's
+    storage type: bf16, or float32 for the float32 path)."""
     s = case.shape
     D, F, V, Hq, Hkv, d = s.hidden, s.ffn, s.vocab, s.n_q_heads, s.n_kv_heads, s.head_dim
     qkv = (Hq + 2 * Hkv) * d
     N, B = case.work.n_requests, case.work.block
-    e = 2
+    e = 2 if s.dtype == "bf16" else 4
     full = kclass.startswith("gemm_full")
     M = N * B if full else R
-    gem = {"qkv": (qkv, D, M * qkv * 4), "o": (D, Hq * d, M * D * 4), "gateup": (2 * F, D, M * F * e),
-           "down": (D, F, M * D * 4), "lmhead": (V, D, 0)}
+    # outputs: q and the cache rows (bf16) for QKV; the float32 residual read and written for O / down;
+    # the SwiGLU activations (bf16) for gate / up; per-tile statistics only (no logits) for the LM head
+    gem = {"qkv": (qkv, D, M * qkv * e), "o": (D, Hq * d, M * D * 8), "gateup": (2 * F, D, M * F * e),
+           "down": (D, F, M * D * 8), "lmhead": (V, D, M * ((V + 127) // 128) * 12)}
     for key, (n, k, out_bytes) in gem.items():
         if kclass.endswith("_" + key) or kclass == "gemm_" + key:
             return n * k * e + M * k * e + out_bytes, 2.0 * M * n * k
@@ -168,6 +171,58 @@ def algorithmic_work(kclass: str, case: fs.Case, R: int, kept_per_req, plen, spl
             fl += 4.0 * rows[b] * Hq * d * keys
         return by, fl
     return None, None
+
+
+def step_work(case: fs.Case, R: int, kept_per_req, plen):
+    """Every launch of one step as (kernel class, launches, algorithmic bytes, flops per launch), in the
+    step's order: embedding + norm; layers 0-1 on all N*B rows (QKV, attention with importance, O,
+    norm, gate/up, down, and a norm between the layers); selection; the norm that gathers the kept rows;
+    layers 2..L-1 on the R kept rows (QKV, ragged attention, O, norm, gate/up, down, norm); LM head;
+    combine + decode.  Norms read the float32 residual and write bf16 rows (the gathering norm also
+    writes the compacted float32 rows)."""
+    s = case.shape
+    L, D = s.n_layers, s.hidden
+    N, B = case.work.n_requests, case.work.block
+    e = 2 if s.dtype == "bf16" else 4
+    rows_full = N * B
+    n_kept_layers = L - 2
+    work = [("embed_norm", 1, rows_full * D * (e + 4 + e), 0.0)]
+    for kc, n in (("gemm_full_qkv", 2), ("attn_score", 2), ("gemm_full_o", 2), ("gemm_full_gateup", 2),
+                  ("gemm_full_down", 2)):
+        by, fl = algorithmic_work(kc, case, R, kept_per_req, plen)
+        work.append((kc, n, by, fl))
+    work.append(("row_norm", 3, rows_full * D * (4 + e), 0.0))
+    work.append(("select", 1, 2 * N * s.n_kv_heads * B * 4 + 2 * N * B, 0.0))
+    work.append(("row_norm", 1, R * D * (4 + 4 + e), 0.0))
+    for kc in ("gemm_qkv", "attn_ragged", "gemm_o", "gemm_gateup", "gemm_down"):
+        by, fl = algorithmic_work(kc, case, R, kept_per_req, plen)
+        work.append((kc, n_kept_layers, by, fl))
+    work.append(("row_norm", 2 * n_kept_layers, R * D * (4 + e), 0.0))
+    by, fl = algorithmic_work("gemm_lmhead", case, R, kept_per_req, plen)
+    work.append(("gemm_lmhead", 1, by, fl))
+    work.append(("decode", 2, R * ((s.vocab + 127) // 128) * 12 + 3 * N * B * 4, 0.0))
+    return work
+
+
+def step_roofline(work, peaks: dict, ms_per_step: float) -> dict:
+    """Sum over the step's launches of max(bytes / HBM peak, flops / sustained bf16 peak), against the
+    measured step time (a step is seconds of back-to-back kernels, so the sustained tensor figure)."""
+    bw, tf = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops_sustained"] * 1e12
+    t_hbm = t_tensor = 0.0
+    total_bytes = total_flops = 0.0
+    for _kc, n, by, fl in work:
+        tb, tt = by / bw, fl / tf
+        if tt > tb:
+            t_tensor += n * tt
+        else:
+            t_hbm += n * tb
+        total_bytes += n * by
+        total_flops += n * fl
+    t_roof_ms = (t_hbm + t_tensor) * 1e3
+    return {"t_roof_ms": t_roof_ms, "measured_ms": ms_per_step,
+            "frac": t_roof_ms / ms_per_step if ms_per_step > 0 else None,
+            "hbm_bound_ms": t_hbm * 1e3, "tensor_bound_ms": t_tensor * 1e3,
+            "algorithmic_gb": total_bytes / 1e9, "algorithmic_tflop": total_flops / 1e12}
 
 
 def source_digest(kclass: str) -> str:
@@ -528,6 +583,10 @@ def main():
                          "algorithmic_bytes_per_launch": by, "algorithmic_flops_per_launch": fl,
                          "kept_rows": R})
 
+    # ---- the whole step against its roofline (sum over launches of the slower of bytes and flops)
+    step_roof = step_roofline(step_work(case, R, kept.tolist(), plen.tolist()), peaks, max_ms / K)
+    step_roof["peak_source"] = f"{peak_src} (HBM copy; sustained bf16)"
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = fs.Case(shp, w, {k: ([x.cpu() for x in v] if isinstance(v, list) else v.cpu())
@@ -556,7 +615,7 @@ def main():
                        "l2": "inputs larger than L2 (3.4 GB of weights and ~2.4 GB of KV pages streamed per step)",
                        "parallelism": f"replicas x{world} (requests sharded, no collective)"},
             "gpu_launches": launches_per_step * K,
-            "clocks": clocks, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clocks, "roofline": roofline, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
             "per_class_ms_per_step": {k: round(v[0], 4) for k, v in per_class.items()} if per_class else None,
         }
         print(json.dumps(line), flush=True)
