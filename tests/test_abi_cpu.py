@@ -88,3 +88,43 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "libfocus.so"))
     with pytest.raises(ImportError):
         _abi.load()
+
+
+def test_null_handles_of_the_block_loop_and_profiling_are_safe():
+    lib = _abi.load()
+    assert lib.focus_commit_block(None, None, None) == _abi.FOCUS_ERR_INVALID_ARG
+    assert lib.focus_decode_block(None, None, None, 4, None, None, None) == _abi.FOCUS_ERR_INVALID_ARG
+    assert lib.focus_last_step_launches(None) == -1
+    assert lib.focus_profile_begin(None, 0, 1) == _abi.FOCUS_ERR_INVALID_ARG
+    assert lib.focus_profile_end(None, None, None) == _abi.FOCUS_ERR_INVALID_ARG
+
+
+# the allocation-free LM head checks its arguments and limits before any device call; the dummy pointers
+# below are never dereferenced on these paths
+_P = C.c_void_p(4096)
+
+
+@pytest.mark.parametrize("rows,dim,vocab,eps,code", [
+    (-1, 2048, 1000, 1e-6, _abi.FOCUS_ERR_INVALID_ARG),
+    (4, 0, 1000, 1e-6, _abi.FOCUS_ERR_INVALID_ARG),
+    (4, 2048, 0, 1e-6, _abi.FOCUS_ERR_INVALID_ARG),
+    (4, 2048, 1000, float("nan"), _abi.FOCUS_ERR_INVALID_ARG),
+    (257, 2048, 1000, 1e-6, _abi.FOCUS_ERR_LIMITS),
+    (4, 4224, 1000, 1e-6, _abi.FOCUS_ERR_LIMITS),
+    (4, 2048, 163841, 1e-6, _abi.FOCUS_ERR_LIMITS),
+    (4, 200, 1000, 1e-6, _abi.FOCUS_ERR_UNSUPPORTED),
+    (0, 2048, 1000, 1e-6, _abi.FOCUS_OK),
+])
+def test_lm_head_noalloc_checks_before_the_device(rows, dim, vocab, eps, code):
+    lib = _abi.load()
+    assert lib.focus_lm_head_conf_noalloc(_P, rows, dim, _P, _P, vocab, eps, _P, _P, None) == code
+
+
+def test_lm_head_noalloc_rejects_null_buffers():
+    lib = _abi.load()
+    for i in range(5):
+        ptrs = [_P] * 5
+        ptrs[i] = None
+        h, nrm, w, conf, top = ptrs
+        assert lib.focus_lm_head_conf_noalloc(h, 4, 2048, nrm, w, 1000, 1e-6, conf, top, None) == \
+            _abi.FOCUS_ERR_INVALID_ARG
