@@ -42,7 +42,12 @@ The pages print no formula.  The readings taken where they are silent:
     confidence (lowest j on ties) decodes;
   * the model layer is a standard pre-norm decoder layer: RMSNorm, grouped-query
     attention with rotate-half RoPE at absolute position P + j, residual,
-    RMSNorm, SwiGLU MLP, residual; a final RMSNorm feeds an untied LM head.
+    RMSNorm, SwiGLU MLP, residual; a final RMSNorm feeds an untied LM head;
+  * around the step (decode_block, commit_block): a block starts with a dense
+    step, focused steps follow until no position is masked, the decoded block is
+    run densely once more, and its K/V then join the prefix pages at positions
+    P .. P + B - 1 (project page, Overview -- Motivation: the prefix is cached
+    exactly).
 
 Parity pins: tests/test_oracle_*.py (closed forms, invariants, brute force,
 an independent dense forward).  Method quality -- whether the delta predicts
