@@ -165,15 +165,25 @@ typedef struct focus_ctx focus_ctx;
 /* Validate the model and limits, record the (borrowed) weight pointers, allocate
  * the workspace and build the TMA descriptors of every weight matrix.  Uses the
  * current CUDA device.  Supported: L >= 2, Hq % Hkv == 0, d in {64, 128} (128 for
- * bf16), D % 128 == 0, F % 64 == 0, B <= 64, max_keep <= max_block.
- * Returns FOCUS_OK and *out, or an error with *out = NULL. */
+ * bf16), D % 128 == 0 and D <= 4096, F % 64 == 0, B <= 64, max_keep <= max_block.
+ * Returns FOCUS_OK and *out, or an error with *out = NULL: FOCUS_ERR_INVALID_ARG (null
+ * pointers, a missing weight, an inconsistent model), FOCUS_ERR_UNSUPPORTED (a shape outside
+ * the list above), FOCUS_ERR_NO_MEMORY (workspace) or FOCUS_ERR_CUDA. */
 int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_limits* lim, focus_ctx** out);
 
 /* Enqueue one focused denoising step on `stream` (a cudaStream_t; NULL = legacy
  * default stream).  No host synchronisation inside; the launch sequence depends
  * only on the host-visible sizes (N, B, parameters), so it can be captured in a
  * CUDA graph.  Outputs are valid once the stream has completed.  Two steps on
- * the same context must not overlap in time (the workspace is shared). */
+ * the same context must not overlap in time (the workspace is shared).  The
+ * device current at the call must be the context's.  N == 0 returns FOCUS_OK and
+ * launches nothing.  Returns FOCUS_ERR_INVALID_ARG (null handle or buffer, N < 0,
+ * B <= 0, k_min > k_max, k_max > B, a NaN tau / threshold, alpha < 0, a forced
+ * fraction above 1, forced_keep_idx without forced_keep_count or the reverse,
+ * another device current), FOCUS_ERR_LIMITS (N, B or the kept bound beyond the
+ * limits), FOCUS_ERR_UNSUPPORTED (a bf16 model with a page size other than 16, 32
+ * or 64) or FOCUS_ERR_CUDA (a launch failed); device-side problems go to the
+ * device error word (see Conventions). */
 int focus_step(focus_ctx* ctx, const focus_batch* in, const focus_params* p, focus_step_out* out, void* stream);
 
 /* ---- around the step: one block to completion --------------------------------
