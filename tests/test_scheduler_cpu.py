@@ -1,0 +1,173 @@
+"""The effective-batch scheduler (continuous batching around the focused step), on the CPU with the oracle
+as its engine.  The step treats requests independently, so whatever the schedule -- arrivals, slot
+reuse, requests in different phases of their block loops sharing an iteration -- every request must
+decode exactly what it decodes alone through the oracle's block loop, and commit exactly the same K/V."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import focus_synth as fs
+from oracle import focus_oracle as fo
+from decodability_aware_token_b200.scheduler import EffectiveBatchScheduler, Request
+
+B = 8          # block size of these runs (the oracle takes any)
+S = 16         # page size
+MAX_PAGES = 6
+
+
+class OracleEngine:
+    """The scheduler's engine with the oracle's step and commit (float64 state, so nothing is rounded
+    between steps and the comparison with the oracle's own block loop is exact)."""
+
+    def __init__(self, case):
+        self.shape, self.model, self.w = case.shape, case.model, case.work
+        self.calls = []
+
+    def step(self, view, dense):
+        w = self.w
+        r = fo.focus_step(self.shape, self.model, view, tau=w.tau, k_min=w.k_min, k_max=w.k_max,
+                          conf_threshold=w.conf_threshold, alpha=w.alpha,
+                          forced_keep_frac=1.0 if dense else -1.0, max_keep=B)
+        view["block_tokens"].copy_(torch.as_tensor(r.block_tokens))
+        view["mask"].copy_(torch.as_tensor(r.mask))
+        view["ibc"].copy_(torch.as_tensor(r.ibc))
+        self.calls.append(("dense" if dense else "focused", view["block_tokens"].shape[0]))
+
+    def commit(self, view):
+        pool, plen = fo.commit_block(view["kv_pool"], view["ibc"], view["prefix_len"], view["page_table"])
+        view["kv_pool"].copy_(torch.as_tensor(pool))
+        view["prefix_len"].copy_(torch.as_tensor(plen))
+        self.calls.append(("commit", 1))
+
+
+def _setup(prompts, seed=7, spare=24):
+    """A float64 page pool holding every request's prompt K/V (N(0,1), seeded) in shuffled pages, plus
+    `spare` free pages; returns (pool, prompt pages per request, free pages)."""
+    case = fs.make_case("tiny")
+    s = case.shape
+    need = [-(-p // S) for p in prompts]
+    n_pages = sum(need) + spare
+    g = torch.Generator().manual_seed(seed)
+    pool = torch.randn(n_pages, s.n_layers, 2, s.n_kv_heads, S, s.head_dim, generator=g, dtype=torch.float64)
+    order = torch.randperm(n_pages, generator=g).tolist()
+    pages, at = [], 0
+    for n in need:
+        pages.append(order[at:at + n])
+        at += n
+    return case, pool, pages, order[at:]
+
+
+def _alone(case, pool, prompt_len, prompt_pages, n_blocks):
+    """Decode one request by itself through the oracle's block loop, block after block."""
+    s, w = case.shape, case.work
+    pool = pool.clone().numpy()
+    used = set(range(pool.shape[0])) - set(prompt_pages)
+    free = sorted(used)
+    pages = list(prompt_pages)
+    plen = prompt_len
+    blocks, steps = [], []
+    for _ in range(n_blocks):
+        while len(pages) * S < plen + B:
+            pages.append(free.pop(0))
+        row = np.full((1, MAX_PAGES), -1, dtype=np.int64)
+        row[0, : len(pages)] = pages
+        batch = {"block_tokens": np.full((1, B), s.vocab - 1), "mask": np.ones((1, B)),
+                 "prefix_len": np.array([plen]), "page_table": row, "kv_pool": pool,
+                 "ibc": np.zeros((1, s.n_layers, 2, s.n_kv_heads, B, s.head_dim))}
+        res = fo.decode_block(s, case.model, batch, tau=w.tau, k_min=w.k_min, k_max=w.k_max,
+                              conf_threshold=w.conf_threshold, alpha=w.alpha)
+        blocks.append(res.block_tokens[0].copy())
+        steps.append(len(res.steps))
+        pool, plen = res.kv_pool, int(res.prefix_len[0])
+    return blocks, steps, _kv(pool, pages, plen)
+
+
+def _kv(pool, pages, plen):
+    """The request's K/V by position: [plen, L, 2, Hkv, d]."""
+    pool = np.asarray(pool)
+    return np.stack([pool[pages[p // S], :, :, :, p % S, :] for p in range(plen)])
+
+
+def _scheduler(case, pool, free, **kw):
+    s = case.shape
+    return EffectiveBatchScheduler(OracleEngine(case), block=B, n_layers=s.n_layers, n_kv_heads=s.n_kv_heads,
+                                   head_dim=s.head_dim, max_pages_per_req=MAX_PAGES, kv_pool=pool, free_pages=free,
+                                   mask_token=s.vocab - 1, k_max=case.work.k_max, **kw)
+
+
+PROMPTS = [24, 0, 40, 16, 7]
+ARRIVALS = [0, 0, 1, 2, 6]
+NBLOCKS = [2, 1, 2, 1, 2]
+
+
+def test_every_request_decodes_what_it_decodes_alone():
+    case, pool, pages, free = _setup(PROMPTS)
+    init = pool.clone()
+    sch = _scheduler(case, pool, free, slots=3, keep_pages=True)
+    for r, (p, a, nb) in enumerate(zip(PROMPTS, ARRIVALS, NBLOCKS)):
+        sch.submit(Request(r, a, p, pages[r], nb))
+    res = sch.run(max_iterations=400)
+    assert sorted(res) == list(range(len(PROMPTS)))
+    for r, (p, nb) in enumerate(zip(PROMPTS, NBLOCKS)):
+        blocks, steps, kv = _alone(case, init, p, pages[r], nb)
+        got = res[r]
+        assert got.prefix_len == p + nb * B
+        assert [b.tolist() for b in got.blocks] == [b.tolist() for b in blocks], f"request {r}"
+        assert got.steps == steps, f"request {r}"
+        np.testing.assert_array_equal(_kv(sch.kv_pool.numpy(), got.pages, got.prefix_len), kv)
+    # the schedule really mixed phases: some iteration ran a focused and a dense call together
+    assert any(st.focused and st.dense for st in sch.stats)
+    assert all(st.active <= 3 for st in sch.stats)
+
+
+def test_slots_and_pages_are_recycled():
+    case, pool, pages, free = _setup(PROMPTS, spare=8)
+    total = len(free) + sum(len(p) for p in pages)
+    sch = _scheduler(case, pool, free, slots=2)
+    for r, (p, a, nb) in enumerate(zip(PROMPTS, ARRIVALS, NBLOCKS)):
+        sch.submit(Request(r, a, p, pages[r], nb))
+    sch.run(max_iterations=400)
+    assert sch.done() and not sch.slot_req
+    assert sorted(sch.free) == list(range(total))          # every page is back in the pool
+    for r, a in enumerate(ARRIVALS):
+        assert sch.results[r].admitted >= a
+    # first come, first served
+    adm = [sch.results[r].admitted for r in range(len(PROMPTS))]
+    assert adm == sorted(adm)
+
+
+def test_row_budget_sets_the_effective_batch():
+    """With the budget of a dense engine on 2 requests (2 x B rows), focused requests (k_max rows each)
+    let more requests run at once than slots counted densely would."""
+    prompts = [16] * 6
+    case, pool, pages, free = _setup(prompts)
+    k_max = 2
+    case = dataclasses.replace(case, work=dataclasses.replace(case.work, k_min=1, k_max=k_max))
+    dense_budget = 2 * B
+    sch = _scheduler(case, pool, free, slots=6, row_budget=dense_budget)
+    for r, p in enumerate(prompts):
+        sch.submit(Request(r, 2 * r, p, pages[r], 1))   # staggered: each arrives while others are focused
+    sch.run(max_iterations=400)
+    # a dense engine with this budget runs 2 requests; focused ones cost k_max rows, so more fit
+    assert max(st.active for st in sch.stats) > dense_budget // B
+    for st in sch.stats:
+        assert st.row_cost == st.focused * k_max + st.dense * B
+    # every admission respected the budget: the iteration that admitted a request stayed within it
+    prev = 0
+    for st in sch.stats:
+        if st.active > prev:
+            assert st.row_cost <= dense_budget
+        prev = st.active
+
+
+def test_requests_that_cannot_fit_are_refused():
+    case, pool, pages, free = _setup([24])
+    sch = _scheduler(case, pool, free, slots=1)
+    with pytest.raises(ValueError):
+        sch.submit(Request(0, 0, 24, pages[0], (MAX_PAGES * S - 24) // B + 1))   # beyond the page table
+    with pytest.raises(ValueError):
+        sch.submit(Request(1, 0, 24, pages[0][:1], 1))                            # prompt pages missing
+    with pytest.raises(ValueError):
+        _scheduler(case, pool, free, slots=1, row_budget=B - 1)
