@@ -171,3 +171,60 @@ def test_requests_that_cannot_fit_are_refused():
         sch.submit(Request(1, 0, 24, pages[0][:1], 1))                            # prompt pages missing
     with pytest.raises(ValueError):
         _scheduler(case, pool, free, slots=1, row_budget=B - 1)
+
+
+class _MarshalOnlyContext:
+    """Stands in for a FocusContext on the CPU: every call goes through the binding's own argument
+    marshalling (dtype, device, contiguity and shape checks, ctypes structs), then the oracle does the
+    work.  It checks that FocusEngine hands the library well-formed slot views and output slices."""
+
+    def __init__(self, case, max_requests):
+        from decodability_aware_token_b200 import _abi
+        self.shape, self.model, self.w = case.shape, case.model, case.work
+        self.dtype, self.device = torch.float64, torch.device("cpu")
+        self.limits = _abi.Limits(max_requests, B, B, MAX_PAGES)
+        self.params_seen = []
+        self.calls = []
+
+    @property
+    def max_keep(self):
+        return self.limits.max_keep
+
+    def alloc_outputs(self, n, block, importance=True, hidden=True):
+        from decodability_aware_token_b200 import FocusContext
+        return FocusContext.alloc_outputs(self, n, block, importance, hidden)
+
+    def step(self, batch, params, out=None, stream=None):
+        from decodability_aware_token_b200 import FocusContext
+        FocusContext._marshal(self, batch, params, out)
+        self.params_seen.append(params.forced_keep_frac)
+        OracleEngine.step(self, batch, dense=params.forced_keep_frac == 1.0)
+
+    def commit_block(self, batch, stream=None):
+        from decodability_aware_token_b200 import FocusContext, StepParams
+        n, block = batch["block_tokens"].shape
+        FocusContext._marshal(self, batch, StepParams(), self.alloc_outputs(n, block))
+        OracleEngine.commit(self, batch)
+
+
+def test_focus_engine_marshals_slot_views_for_the_library():
+    from decodability_aware_token_b200 import StepParams
+    from decodability_aware_token_b200.scheduler import FocusEngine
+    case, pool, pages, free = _setup(PROMPTS)
+    init = pool.clone()
+    w = case.work
+    ctx = _MarshalOnlyContext(case, max_requests=3)
+    params = StepParams(w.tau, w.k_min, w.k_max, w.conf_threshold, w.alpha)
+    s = case.shape
+    sch = EffectiveBatchScheduler(FocusEngine(ctx, params), slots=3, block=B, n_layers=s.n_layers,
+                                  n_kv_heads=s.n_kv_heads, head_dim=s.head_dim, max_pages_per_req=MAX_PAGES,
+                                  kv_pool=pool, free_pages=free, mask_token=s.vocab - 1, k_max=w.k_max,
+                                  keep_pages=True)
+    for r, (p, a, nb) in enumerate(zip(PROMPTS, ARRIVALS, NBLOCKS)):
+        sch.submit(Request(r, a, p, pages[r], nb))
+    res = sch.run(max_iterations=400)
+    assert set(ctx.params_seen) == {1.0, -1.0}          # dense and focused calls, nothing else
+    for r, (p, nb) in enumerate(zip(PROMPTS, NBLOCKS)):
+        blocks, _, kv = _alone(case, init, p, pages[r], nb)
+        assert [b.tolist() for b in res[r].blocks] == [b.tolist() for b in blocks]
+        np.testing.assert_array_equal(_kv(sch.kv_pool.numpy(), res[r].pages, res[r].prefix_len), kv)
