@@ -17,7 +17,7 @@ requests leave their slot at once and waiting ones take it (continuous batching)
 
 Admission (the effective batch): a request in a focused step costs at most k_max rows in layers
 2..L-1, one in a dense step costs B.  A waiting request is admitted while a slot is free, the pages for
-its next block are available, and the summed cost of the active requests plus B (its dense first step)
+all its blocks can be reserved, and the summed cost of the active requests plus B (its dense first step)
 stays within ``row_budget``.  A dense engine spending N x B rows per step admits N requests; with the
 same budget, focused requests cost k_max, so up to N x B / k_max of them run at once.
 
@@ -151,6 +151,10 @@ class EffectiveBatchScheduler:
         """Pages to add so that positions up to prefix + B are mapped."""
         return max(0, -(-(rec["prefix_len"] + self.B) // self.page_size) - len(rec["pages"]))
 
+    def _pages_for_request(self, req: Request) -> int:
+        """Pages a request needs beyond its prompt pages to hold all its blocks."""
+        return max(0, -(-(req.prompt_len + req.n_blocks * self.B) // self.page_size) - len(req.prompt_pages))
+
     def _cost(self, rec: dict) -> int:
         return self.k_max if rec["phase"] == _FOCUSED else self.B
 
@@ -163,21 +167,24 @@ class EffectiveBatchScheduler:
         self.page_table[i].copy_(row)
 
     def _start_block(self, rec: dict) -> None:
-        need = self._pages_needed(rec)
-        rec["pages"].extend(self.free[:need])
-        del self.free[:need]
+        need = self._pages_needed(rec)  # taken from the pages reserved at admission
+        rec["pages"].extend(rec["reserved"][:need])
+        del rec["reserved"][:need]
         rec["phase"] = _DENSE_FIRST
         rec["block_steps"] = 0
 
     def _admit(self) -> None:
         while self.waiting and self.waiting[0].arrival <= self.iteration and len(self.slot_req) < self.slots:
             req = self.waiting[0]
-            rec = {"req": req, "prefix_len": req.prompt_len, "pages": list(req.prompt_pages), "blocks": [],
-                   "steps": [], "admitted": self.iteration}
             cost = sum(self._cost(r) for r in self.slot_req)
-            if cost + self.B > self.row_budget or self._pages_needed(rec) > len(self.free):
+            need = self._pages_for_request(req)
+            if cost + self.B > self.row_budget or need > len(self.free):
                 break  # first come, first served: nobody overtakes the head of the queue
             self.waiting.pop(0)
+            # every page the request will need is reserved now, so no request stalls mid-flight
+            rec = {"req": req, "prefix_len": req.prompt_len, "pages": list(req.prompt_pages), "blocks": [],
+                   "steps": [], "admitted": self.iteration, "reserved": self.free[:need]}
+            del self.free[:need]
             self._start_block(rec)
             self.slot_req.append(rec)
             self._write_slot(len(self.slot_req) - 1, rec)
@@ -235,8 +242,6 @@ class EffectiveBatchScheduler:
                 rec["steps"].append(rec["block_steps"])
                 rec["prefix_len"] += self.B
                 if len(rec["blocks"]) < rec["req"].n_blocks:
-                    if self._pages_needed(rec) > len(self.free):
-                        raise RuntimeError("page pool exhausted while a request is in flight")
                     self._start_block(rec)
                     self._write_slot(i, rec)
                 else:
@@ -256,6 +261,7 @@ class EffectiveBatchScheduler:
                                                   rec["prefix_len"], list(rec["pages"]), rec["steps"])
             if not self.keep_pages:
                 self.free.extend(rec["pages"])
+            self.free.extend(rec["reserved"])  # none left once every block is placed
         st = IterationStats(self.iteration, n, n_f, n - n_f, cost, committed)
         self.stats.append(st)
         self.iteration += 1

@@ -228,3 +228,16 @@ def test_focus_engine_marshals_slot_views_for_the_library():
         blocks, _, kv = _alone(case, init, p, pages[r], nb)
         assert [b.tolist() for b in res[r].blocks] == [b.tolist() for b in blocks]
         np.testing.assert_array_equal(_kv(sch.kv_pool.numpy(), res[r].pages, res[r].prefix_len), kv)
+
+
+def test_admission_reserves_every_page_a_request_needs():
+    """A pool with room for one long request at a time: the second waits for the first to finish
+    instead of starting and running out of pages mid-flight."""
+    prompts = [16, 16]
+    case, pool, pages, free = _setup(prompts, spare=3)            # 3 free pages: 3 blocks of 8 over 16 tokens
+    sch = _scheduler(case, pool, free, slots=2)
+    sch.submit(Request(0, 0, 16, pages[0], 3))                     # needs ceil((16 + 24) / 16) - 1 = 2 pages
+    sch.submit(Request(1, 0, 16, pages[1], 3))                     # 2 more: only 1 left while 0 runs
+    res = sch.run(max_iterations=400)
+    assert res[1].admitted > res[0].admitted
+    assert res[1].admitted >= res[0].finished
