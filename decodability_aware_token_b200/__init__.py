@@ -223,6 +223,13 @@ class FocusContext:
                                                 C.byref(steps), C.c_void_p(s.cuda_stream)), "focus_decode_block")
         return out, int(steps.value)
 
+    def probe_wait_timeout(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """Enqueue the failure-path probe: a bounded pipeline wait that nothing satisfies gives up after
+        about a second and flags FOCUS_DEVERR_TIMEOUT (read it with device_error)."""
+        with torch.cuda.device(self.device):
+            s = stream if stream is not None else torch.cuda.current_stream(self.device)
+            _check(self._lib.focus_probe_wait_timeout(self._ctx, C.c_void_p(s.cuda_stream)), "focus_probe_wait_timeout")
+
     def last_step_launches(self) -> int:
         """Kernels the most recent step enqueued."""
         return int(self._lib.focus_last_step_launches(self._ctx))

@@ -25,7 +25,7 @@ FOCUS_DTYPE_BF16 = 1
 # every symbol include/focus.h declares (checked by the CPU tests)
 EXPORTED = ("focus_init", "focus_step", "focus_destroy", "focus_status_string", "focus_get_device_error",
             "focus_workspace_bytes", "focus_last_step_launches", "focus_profile_begin", "focus_profile_end",
-            "focus_lm_head_conf_noalloc", "focus_commit_block", "focus_decode_block")
+            "focus_lm_head_conf_noalloc", "focus_commit_block", "focus_decode_block", "focus_probe_wait_timeout")
 
 KERNEL_CLASSES = ("embed_norm", "qkv_finalize", "attn_score", "attn_ragged", "row_norm", "select", "decode",
                   "gemm_full_qkv", "gemm_full_o", "gemm_full_gateup", "gemm_full_down",
@@ -100,6 +100,8 @@ def load():
     lib.focus_lm_head_conf_noalloc.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_int32,
                                                C.c_float, C.c_void_p, C.c_void_p, C.c_void_p]
     lib.focus_lm_head_conf_noalloc.restype = C.c_int
+    lib.focus_probe_wait_timeout.argtypes = [C.c_void_p, C.c_void_p]
+    lib.focus_probe_wait_timeout.restype = C.c_int
     lib.focus_commit_block.argtypes = [C.c_void_p, C.POINTER(Batch), C.c_void_p]
     lib.focus_commit_block.restype = C.c_int
     lib.focus_decode_block.argtypes = [C.c_void_p, C.POINTER(Batch), C.POINTER(Params), C.c_int32, C.POINTER(StepOut),

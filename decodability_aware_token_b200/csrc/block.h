@@ -18,5 +18,8 @@ struct CommitArgs {
 int launch_commit_block(const CommitArgs& a, cudaStream_t s);
 // Number of nonzero bytes in mask[0 .. n) into *out (one launch).
 int launch_count_masked(const uint8_t* mask, int n, int32_t* out, cudaStream_t s);
+// One CTA whose bounded pipeline wait is never satisfied: sets FOCUS_DEVERR_TIMEOUT in *err after about a
+// second and returns (probe.cu); returns the launch count or -1.
+int launch_wait_timeout_probe(int* err, cudaStream_t s);
 
 }  // namespace focus

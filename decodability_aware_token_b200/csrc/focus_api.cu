@@ -616,6 +616,13 @@ int focus_get_device_error(focus_ctx* c, int32_t* bits) {
     return v ? FOCUS_ERR_DEVICE_BOUNDS : FOCUS_OK;
 }
 
+int focus_probe_wait_timeout(focus_ctx* c, void* stream) {
+    if (!c) return FOCUS_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != c->device) return FOCUS_ERR_INVALID_ARG;
+    return launch_wait_timeout_probe(c->err, static_cast<cudaStream_t>(stream)) == 1 ? FOCUS_OK : FOCUS_ERR_CUDA;
+}
+
 int focus_last_step_launches(const focus_ctx* c) { return c ? c->last_launches : -1; }
 
 int focus_profile_begin(focus_ctx* c, int kernel_class, int max_launches) {

@@ -226,6 +226,14 @@ const char* focus_status_string(int status);
  * FOCUS_ERR_DEVICE_BOUNDS; *bits (if not NULL) receives the raw FOCUS_DEVERR_* bits. */
 int focus_get_device_error(focus_ctx* ctx, int32_t* bits);
 
+/* Failure-path probe (no counterpart in the paper): enqueue one CTA whose pipeline wait -- the same
+ * bounded mbarrier wait the GEMM and attention kernels use -- is never satisfied.  After about a second
+ * the wait gives up, sets FOCUS_DEVERR_TIMEOUT in the context's device error word and the kernel
+ * returns, so focus_get_device_error then reports FOCUS_ERR_TIMEOUT and the context stays usable (no
+ * trap, no fault).  For health checks of the failure path.  The device current at the call must be
+ * the context's.  Returns FOCUS_OK, FOCUS_ERR_INVALID_ARG or FOCUS_ERR_CUDA. */
+int focus_probe_wait_timeout(focus_ctx* ctx, void* stream);
+
 /* Size in bytes of the workspace a context with these limits allocates (0 on bad arguments). */
 size_t focus_workspace_bytes(const focus_model_cfg* cfg, const focus_limits* lim);
 

@@ -97,6 +97,7 @@ def test_null_handles_of_the_block_loop_and_profiling_are_safe():
     assert lib.focus_last_step_launches(None) == -1
     assert lib.focus_profile_begin(None, 0, 1) == _abi.FOCUS_ERR_INVALID_ARG
     assert lib.focus_profile_end(None, None, None) == _abi.FOCUS_ERR_INVALID_ARG
+    assert lib.focus_probe_wait_timeout(None, None) == _abi.FOCUS_ERR_INVALID_ARG
 
 
 # the allocation-free LM head checks its arguments and limits before any device call; the dummy pointers

@@ -143,6 +143,25 @@ def test_prefix_beyond_page_table_is_clamped_and_flagged():
     assert gpu["device_bits"] & _abi.FOCUS_DEVERR_PREFIX
 
 
+def test_bounded_wait_expires_with_a_timeout_status_and_the_context_stays_usable():
+    """Failure detection without a fault: a pipeline wait that nothing satisfies gives up after about a
+    second, the error word says so, and the same context then runs a clean step."""
+    from decodability_aware_token_b200 import FocusContext, _abi
+    case = _case("tiny")
+    m = _model("tiny", case)
+    p = step_params(case.work)
+    lim = limits_for(case, p)
+    batch = {k: v.cuda().clone() for k, v in case.batch.items()}
+    with FocusContext(case.shape, m, **lim) as ctx:
+        ctx.probe_wait_timeout()
+        rc, bits = ctx.device_error()
+        assert rc == _abi.FOCUS_ERR_TIMEOUT and bits & _abi.FOCUS_DEVERR_TIMEOUT
+        from decodability_aware_token_b200 import StepParams
+        ctx.step(batch, StepParams(**p))
+        rc, bits = ctx.device_error()
+        assert rc == _abi.FOCUS_OK and bits == 0
+
+
 def test_host_validation_rejects_bad_arguments():
     from decodability_aware_token_b200 import FocusContext, StepParams, FocusError, _abi
     case = _case("tiny")
