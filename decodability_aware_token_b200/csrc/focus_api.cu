@@ -14,6 +14,8 @@
 #include <new>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>  // header-only; ranges are no-ops unless a profiler is attached
+
 #include "launch.h"
 #include "tc_gemm.h"
 #include "block.h"
@@ -57,6 +59,13 @@ struct focus_ctx {
 namespace {
 
 constexpr int kMaxSplits = 8;
+
+// NVTX range names, one per focus_kernel_class (profilers group the step's launches by these)
+const char* const kClassNames[] = {"embed_norm", "qkv_finalize", "attn_score", "attn_ragged", "row_norm",
+                                   "select", "decode", "gemm_full_qkv", "gemm_full_o", "gemm_full_gateup",
+                                   "gemm_full_down", "gemm_qkv", "gemm_o", "gemm_gateup", "gemm_down",
+                                   "gemm_lmhead"};
+static_assert(sizeof(kClassNames) / sizeof(kClassNames[0]) == FOCUS_K_COUNT, "one name per kernel class");
 
 struct Layout {
     size_t off[32];
@@ -186,6 +195,7 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
     if (c->prof_active) FOCUS_CUDA_TRY(cudaStreamIsCapturing(s, &cap));
     const unsigned rec_flags = cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
     auto run = [&](int kclass, auto&& launch) {
+        nvtxRangePushA(kClassNames[kclass]);
         const bool timed = c->prof_active && c->prof_class == kclass && c->prof_n < c->prof_cap;
         if (timed && cudaEventRecordWithFlags(c->prof_ev[2 * c->prof_n], s, rec_flags) != cudaSuccess)
             launch_failed = true;
@@ -197,6 +207,7 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
                 launch_failed = true;
             ++c->prof_n;
         }
+        nvtxRangePop();
     };
     auto gemm = [&](int kclass, Epi epi, const void* A, const void* Bw, const void* B2, int Mb, const int32_t* Md,
                     int Nn, int K, int splits, void* act_out, float* resid = nullptr, int layer = 0,
@@ -515,8 +526,11 @@ int focus_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev != c->device) return FOCUS_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (c->cfg.dtype == FOCUS_DTYPE_BF16) return run_step<bf16>(c, in, p, out, s, k_cap);
-    return run_step<float>(c, in, p, out, s, k_cap);
+    nvtxRangePushA("focus_step");
+    const int rc = c->cfg.dtype == FOCUS_DTYPE_BF16 ? run_step<bf16>(c, in, p, out, s, k_cap)
+                                                    : run_step<float>(c, in, p, out, s, k_cap);
+    nvtxRangePop();
+    return rc;
 }
 
 int focus_commit_block(focus_ctx* c, const focus_batch* in, void* stream) {
