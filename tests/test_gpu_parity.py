@@ -6,7 +6,6 @@ checked on sampled requests (requests are independent, so the oracle can run a s
 import dataclasses
 import gc
 
-import numpy as np
 import pytest
 import torch
 
