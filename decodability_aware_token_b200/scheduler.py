@@ -81,6 +81,14 @@ class FocusEngine:
         self.stream = stream
         self._out = None
 
+    def capacity_check(self, slots: int, block: int) -> None:
+        """The context must take every slot in one call and keep all B positions in the dense steps."""
+        lim = self.ctx.limits
+        if slots > lim.max_requests:
+            raise ValueError(f"{slots} slots exceed the context's max_requests ({lim.max_requests})")
+        if block > lim.max_block or block > lim.max_keep:
+            raise ValueError(f"block {block}: the context needs max_block and max_keep >= B for the dense steps")
+
     def _outputs(self, n: int, block: int):
         if self._out is None or self._out.keep_count.shape[0] < n or self._out.decoded_ids.shape[1] != block:
             self._out = self.ctx.alloc_outputs(max(n, 1), block, importance=False, hidden=False)
@@ -112,6 +120,9 @@ class EffectiveBatchScheduler:
                  row_budget: Optional[int] = None, keep_pages: bool = False):
         if slots < 1 or block < 1 or k_max < 1 or max_pages_per_req < 1:
             raise ValueError("slots, block, k_max and max_pages_per_req must be positive")
+        check = getattr(engine, "capacity_check", None)
+        if check is not None:
+            check(slots, block)
         self.engine = engine
         self.slots, self.B, self.k_max = slots, block, min(k_max, block)
         self.page_size = int(kv_pool.shape[4])

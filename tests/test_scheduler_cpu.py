@@ -252,3 +252,20 @@ def test_admission_reserves_every_page_a_request_needs():
     res = sch.run(max_iterations=400)
     assert res[1].admitted > res[0].admitted
     assert res[1].admitted >= res[0].finished
+
+
+def test_focus_engine_refuses_a_context_too_small_for_the_slots_or_block():
+    from decodability_aware_token_b200 import StepParams
+    from decodability_aware_token_b200.scheduler import FocusEngine
+    case, pool, pages, free = _setup([16])
+    s = case.shape
+    eng = FocusEngine(_MarshalOnlyContext(case, max_requests=2), StepParams())
+    kw = dict(block=B, n_layers=s.n_layers, n_kv_heads=s.n_kv_heads, head_dim=s.head_dim, max_pages_per_req=MAX_PAGES,
+              kv_pool=pool, free_pages=free, mask_token=s.vocab - 1, k_max=2)
+    with pytest.raises(ValueError):
+        EffectiveBatchScheduler(eng, slots=3, **kw)                       # more slots than max_requests
+    small = _MarshalOnlyContext(case, max_requests=2)
+    small.limits.max_keep = B // 2
+    with pytest.raises(ValueError):
+        EffectiveBatchScheduler(FocusEngine(small, StepParams()), slots=2, **kw)   # dense steps need max_keep >= B
+    EffectiveBatchScheduler(eng, slots=2, **kw)                           # fits
