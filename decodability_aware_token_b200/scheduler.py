@@ -23,8 +23,9 @@ same budget, focused requests cost k_max, so up to N x B / k_max of them run at 
 
 Readings (the pages describe no scheduler): first come, first served among arrived requests; a
 request's prompt pages and the pages allocated for its blocks return to the pool when it finishes
-(unless ``keep_pages``); every request's results equal those of decoding it alone, since the step
-treats requests independently.
+(unless ``keep_pages``).  The step treats requests independently, so every request decodes what it
+decodes alone: exactly with the oracle as engine; on the GPU up to the float summation order, since the
+attention splits long key walks into pieces only when a batch has few (request, head) units.
 """
 from __future__ import annotations
 
