@@ -142,7 +142,7 @@ class EffectiveBatchScheduler:
         self.page_table = torch.full((slots, max_pages_per_req), -1, dtype=torch.int32, device=dev)
         self.ibc = torch.zeros(slots, n_layers, 2, n_kv_heads, block, head_dim, dtype=kv_pool.dtype, device=dev)
         self.waiting: List[Request] = []
-        self.slot_req: List[Optional[dict]] = []     # per active slot: the request's host-side record
+        self.slot_req: List[dict] = []               # per active slot: the request's host-side record
         self.results: Dict[int, RequestResult] = {}
         self.stats: List[IterationStats] = []
         self.iteration = 0
