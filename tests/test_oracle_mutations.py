@@ -93,6 +93,38 @@ def _layer_variant(write_cache_first=True, mlp_residual=True):
     return layer
 
 
+def _storage_variant(round_residual=False, round_attention_output=True, round_q_after_rope=True):
+    """The oracle's layer with one slip in where bf16 storage rounds (the float64 mode is unaffected)."""
+    def layer(x, lw, shape, positions, rows, prefix_k, prefix_v, cache_k, cache_v, store=fo._keep):
+        hq, hkv, d = shape.n_q_heads, shape.n_kv_heads, shape.head_dim
+        n = x.shape[0]
+        h = store(fo.rms_norm(x, lw["attn_norm"], shape.rms_eps))
+        qkv = h @ lw["wqkv"].T
+        q = qkv[:, : hq * d].reshape(n, hq, d).transpose(1, 0, 2)
+        k = qkv[:, hq * d:(hq + hkv) * d].reshape(n, hkv, d).transpose(1, 0, 2)
+        v = qkv[:, (hq + hkv) * d:].reshape(n, hkv, d).transpose(1, 0, 2)
+        pos = positions[rows]
+        if round_q_after_rope:
+            q = store(fo.rope(q, pos, shape.rope_theta))
+        else:
+            q = fo.rope(store(q), pos, shape.rope_theta)                          # slip: rounds before RoPE
+        k = store(fo.rope(k, pos, shape.rope_theta))
+        cache_k[:, rows] = k
+        cache_v[:, rows] = store(v)
+        keys = np.concatenate([prefix_k, cache_k], axis=1)
+        vals = np.concatenate([prefix_v, cache_v], axis=1)
+        o, p = fo.attention(q, keys, vals)
+        o = store(o) if round_attention_output else o                             # slip: output not rounded
+        x = x + o.transpose(1, 0, 2).reshape(n, hq * d) @ lw["wo"].T
+        if round_residual:
+            x = store(x)                                                          # slip: residual rounded
+        h2 = store(fo.rms_norm(x, lw["mlp_norm"], shape.rms_eps))
+        a = store(fo.silu(h2 @ lw["wgate"].T) * (h2 @ lw["wup"].T))
+        x = x + a @ lw["wdown"].T
+        return (store(x) if round_residual else x), p
+    return layer
+
+
 def _lm_head_highest_id(x, g, w, eps, store=fo._keep):
     conf, top, lc, mg = _orig["lm_head_conf"](x, g, w, eps, store)
     z = fo.rms_norm(x, g, eps) @ w.T
@@ -178,6 +210,9 @@ MUTATIONS = {
     "compaction_descending": ("compact_rows", _compact_descending),
     "fallback_may_pick_unmasked": ("threshold_decode", _decode_fallback_any),
     "fallback_higher_position_on_ties": ("threshold_decode", _decode_fallback_high_j),
+    "bf16_storage_rounds_the_residual": ("layer_forward", _storage_variant(round_residual=True)),
+    "bf16_storage_skips_the_attention_output": ("layer_forward", _storage_variant(round_attention_output=False)),
+    "bf16_storage_rounds_q_before_rope": ("layer_forward", _storage_variant(round_q_after_rope=False)),
 }
 
 PINS = [getattr(pins, n) for n in sorted(dir(pins)) if n.startswith("test_") and n not in (

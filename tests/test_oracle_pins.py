@@ -292,6 +292,22 @@ def test_forced_full_keep_equals_dense_forward(name):
     np.testing.assert_allclose(r.conf.reshape(-1), 1.0 / np.exp(z - z.max(1, keepdims=True)).sum(1), rtol=1e-10)
 
 
+def test_bf16_storage_points_match_an_independent_bf16_forward():
+    """storage='bf16' rounds where the bf16 kernels store activations -- the normalised rows, q and k after
+    RoPE, v, the attention output, the SwiGLU product, the row normalised for the LM head -- and nowhere
+    else (never the residual stream): with every position kept it equals an independently written forward
+    that rounds at exactly those points and accumulates in float64."""
+    case = fs.make_case("tiny")
+    r = _step(case, forced_keep_frac=1.0, storage="bf16")
+    ref = dense_block_forward(case.shape, case.model, case.batch, storage="bf16")
+    N, B = case.batch["block_tokens"].shape
+    np.testing.assert_allclose(r.hidden, ref["hidden"].reshape(N * B, -1).numpy(), rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(r.importance, ref["colsum"].numpy(), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(r.ibc, ref["kv"].numpy(), rtol=1e-9, atol=1e-9)
+    z = ref["logits"].reshape(N * B, -1).numpy()
+    np.testing.assert_allclose(r.conf.reshape(-1), 1.0 / np.exp(z - z.max(1, keepdims=True)).sum(1), rtol=1e-9)
+
+
 def test_page_permutation_leaves_the_step_unchanged():
     case = fs.make_case("small_f32")
     r1 = _step(case)
