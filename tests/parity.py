@@ -1,24 +1,36 @@
 """Tie-aware comparison of a GPU focused step against the CPU oracle.
 
-The oracle here takes its decisions in the kernel's precision: for the bf16 path it rounds activations
-to bf16 where the kernel stores them (oracle storage "bf16"); the float32 path is compared with the
-plain float64 oracle.  (The bf16 path is also checked against the exact float64 oracle, see
-gpu_harness.accuracy_check.)
+Which oracle a case is compared with:
+  * the float32 path, and the bf16 path on shallow models (at most 4 layers): the plain float64 oracle,
+    for values and decisions alike, with no allowance;
+  * the bf16 path on deep models (the 28- and 36-layer shapes): values against the float64 oracle with
+    an allowance of twice the drift that bf16 storage alone causes (see below), decisions against the
+    oracle run with bf16 storage at the kernel's storage points ("decision oracle"); agreement of the
+    decisions with the float64 oracle at 1e-3 gates is counted and reported (decision_report).
+
+Why the deep bf16 cases carry the drift allowance: deep random-weight stacks amplify bf16-level
+perturbations.  tests/test_bf16_drift_cpu.py shows on 28- and 36-layer models with the per-layer gain of
+the 1.7B and 8B shapes that an independently written bf16 evaluation (float32 accumulation, bf16
+probabilities before P.V) lies as far from float64 as the oracle's bf16 mode does (3.7-9 % of RMS
+max-abs, above the 2e-2 bound), that the two differ from each other by about that drift, and that
+2e-2 x RMS plus twice the drift covers the independent one.  At 4 layers the same test shows the strict
+bound holds without any allowance.
 
 Rules (what is unique is compared exactly, what is not is checked for validity):
   * importance, hidden states, confidences: max-abs error <= frac x RMS of the oracle's values
-    (frac = 2e-2 for bf16, 1e-4 for the float32 path), plus, for bf16, twice the drift that bf16
-    storage alone causes (bf16-storage oracle minus float64 oracle, measured per quantity): deep
-    random-weight stacks amplify bf16-level perturbations, so two equally valid bf16 evaluations that
-    differ only in summation order already differ by about that drift (4.2% of RMS at 28 layers);
-    likewise the RMS of the error stays within frac x RMS plus twice the RMS of that drift (the
-    8B shape's 36 layers give confidences a bf16 drift of several % RMS);
+    (frac = 2e-2 for bf16, 1e-4 for the float32 path), plus, for deep bf16 cases, twice the max-abs
+    drift of bf16 storage (bf16-storage oracle minus float64 oracle, per quantity); the RMS of the error
+    <= frac x RMS plus, for deep bf16 cases, twice the RMS of that drift;
   * kept set per request: identical wherever the oracle's delta gap at the top-k cut and its
-    |delta - tau| both exceed the selection gate; otherwise the GPU set must still be a valid top-k of
-    the oracle's deltas within that gate (and the test then re-runs the GPU with the oracle's set
-    forced to compare everything downstream);
+    |delta - tau| both exceed the selection gate (1e-3); otherwise the GPU set must still be a valid
+    top-k of the oracle's deltas within that gate (and the test then re-runs the GPU with the oracle's
+    set forced to compare everything downstream);
   * top id per kept row: identical where the oracle's top-1 logit margin exceeds the logit gate;
-    otherwise the GPU's id must be within the gate of the oracle's best logit;
+    otherwise the GPU's id must be within the gate of the oracle's best logit.  For bf16 the gate is the
+    logit error that the hidden-state tolerance allows (frac x sqrt(D) x RMS of the LM-head weights,
+    about 9e-3 at D = 512): a 1e-3 gate is finer than bf16 storage resolves (an independent bf16
+    evaluation flips a row with a 2.1e-3 margin, tests/test_bf16_drift_cpu.py), so rows between the two
+    gates are counted in decision_report rather than failed;
   * decoded positions / ids: identical where no threshold or fallback decision is within its gate;
   * the intra-block KV cache: rewritten entries within tolerance, every other entry bit-identical.
 """
@@ -225,3 +237,35 @@ def compare(case, params: dict, ora: fo.OracleResult, gpu: dict, tol: Tol, ibc_i
           allow.get("ibc_rms", 0.0))
     assert np.array_equal(ibc_g[~w_idx], ibc0[~w_idx]), "an evicted position's cache entry changed"
     return report, []
+
+
+def decision_report(ora64: fo.OracleResult, gpu: dict, gate: float = 1e-3) -> dict:
+    """Agreement of the GPU's decisions with the plain float64 oracle at `gate` (counts only, no assert).
+
+    kept sets: per request, equal / differing with both of the oracle's selection gaps above the gate
+    ("outside") / differing inside the gate.  top ids: per kept row of the requests whose sets agree,
+    equal / differing with the oracle's top-1 logit margin above the gate / inside it."""
+    kc, ret = _np(gpu["keep_count"]), _np(gpu["retained_idx"])
+    top_g = _np(gpu["top_id"])
+    n = ora64.keep_count.shape[0]
+    rep = dict(gate=gate, requests=n, kept_equal=0, kept_differ_outside=0, kept_differ_inside=0,
+               requests_inside_gate=0, rows=0, top_equal=0, top_differ_outside=0, top_differ_inside=0,
+               rows_inside_gate=0)
+    for b in range(n):
+        kg = ret[b, : kc[b]].tolist()
+        ko = ora64.retained_idx[b, : ora64.keep_count[b]].tolist()
+        inside = not (ora64.cut_gap[b] > gate and ora64.tau_gap[b] > gate)
+        rep["requests_inside_gate"] += int(inside)
+        if kg != ko:
+            rep["kept_differ_inside" if inside else "kept_differ_outside"] += 1
+            continue
+        rep["kept_equal"] += 1
+        for t in range(kc[b]):
+            rep["rows"] += 1
+            near = ora64.logit_margin[b, t] <= gate
+            rep["rows_inside_gate"] += int(near)
+            if top_g[b, t] == ora64.top_id[b, t]:
+                rep["top_equal"] += 1
+            else:
+                rep["top_differ_inside" if near else "top_differ_outside"] += 1
+    return rep
