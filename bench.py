@@ -1,14 +1,16 @@
 #!/usr/bin/env python
 """Throughput of one FOCUS focused denoising step on B200: decoded tokens/s, step latency, roofline.
 
-    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
 
 One "step" is one pass of the whole focused step (embed, layers 0-1 with importance, delta / budget /
 top-k, compaction, layers 2..L-1 on the kept rows, LM head + decode) over one batch.  The default
-workload is the SDAR-1.7B-shaped random-init bf16 model with 32 ragged requests, block 32, prefixes
-U[256, 1024] in 64-token pages, masked fraction U[0.3, 1.0], k_max 8.  Under torchrun each rank runs an
-independent replica on its own 32 requests (requests are independent: no collective on the data
-path), so the scaling is weak.
+workload is the largest one-GPU configuration: the SDAR-8B-shaped random-init bf16 model (36 layers,
+hidden 4096, 32 / 8 heads) with 256 ragged requests, block 64, prefixes U[512, 2048] in 64-token pages,
+masked fraction U[0.3, 1.0], k_max 16.  Other workloads: sdar1.7b_n32_b32, sdar1.7b_n128_b32 and the
+kernel-sweep points sweep_n{N}_b{B}_f{f} (1.7B shape, forced keep fraction f, prefixes U[256, 4096]).
+Under torchrun each rank runs an independent replica on its own requests (requests are independent: no
+collective on the data path), so the scaling is weak.
 
 `--impl reference` times the CPU oracle (test infrastructure, float64 numpy) on the host cores instead,
 one request of the same workload per step.
@@ -21,6 +23,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -46,9 +49,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["focus", "reference"], default="focus")
-    ap.add_argument("--workload", default="sdar1.7b_n32_b32")
+    ap.add_argument("--workload", default="sdar8b_n256_b64",
+                    help="named workload, or sweep_n{N}_b{B}_f{f} for a kernel-sweep point")
     ap.add_argument("--roofline-kernel", default="auto", help="kernel class for the roofline (default: dominant)")
-    ap.add_argument("--cpu-baseline-requests", type=int, default=8)
+    ap.add_argument("--cpu-baseline-requests", type=int, default=None,
+                    help="requests the CPU oracle baseline runs (default: about 20 s of float64 work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager focus_step calls instead of graph replays")
@@ -60,14 +65,23 @@ def parse():
     return ap.parse_args()
 
 
-def make_workload(args, seed, device):
+def resolve_workload(name: str):
+    """(model shape, workload, base seed) of a named workload or of a sweep point sweep_n{N}_b{B}_f{f}."""
+    m = re.fullmatch(r"sweep_n(\d+)_b(\d+)_f([0-9.]+)", name)
+    if m:
+        return (fs.MODEL_SHAPES["sdar1.7b"], fs.sweep_workload(int(m[1]), int(m[2]), float(m[3])), fs.SEEDS["sweep"])
+    sname, wname = fs.CASES[name]
+    return fs.MODEL_SHAPES[sname], fs.WORKLOADS[wname], fs.SEEDS.get(name, 1234)
+
+
+def make_workload(args, seed, device, requests=None):
     """The named workload, optionally with fewer layers / other request counts for small profiling cases."""
-    sname, wname = fs.CASES[args.workload]
-    shape, work = fs.MODEL_SHAPES[sname], fs.WORKLOADS[wname]
+    shape, work, _ = resolve_workload(args.workload)
     if args.layers is not None:
         shape = dataclasses.replace(shape, n_layers=args.layers)
-    if args.requests is not None:
-        work = dataclasses.replace(work, n_requests=args.requests)
+    n = requests if requests is not None else args.requests
+    if n is not None:
+        work = dataclasses.replace(work, n_requests=n)
     return fs.make_case(args.workload, seed=seed, device=device, shape=shape, work=work)
 
 
@@ -224,6 +238,41 @@ def step_roofline(work, peaks: dict, ms_per_step: float) -> dict:
             "algorithmic_gb": total_bytes / 1e9, "algorithmic_tflop": total_flops / 1e12}
 
 
+# kernel families: the launches of one role in the step, whichever kernel runs them (the kept-row GEMMs
+# run on the swapped few-row kernel up to 256 kept rows and on the row-major kernel above)
+FAMILIES = {
+    "gemm_kept_rows": ("gemm_qkv", "gemm_o", "gemm_gateup", "gemm_down"),
+    "gemm_full_block": ("gemm_full_qkv", "gemm_full_o", "gemm_full_gateup", "gemm_full_down"),
+    "gemm_lm_head": ("gemm_lmhead",),
+    "attention_ragged": ("attn_ragged",),
+    "attention_scoring": ("attn_score",),
+    "norms": ("embed_norm", "row_norm", "qkv_finalize"),
+    "select_compact": ("select",),
+    "decode": ("decode",),
+}
+
+
+def family_rooflines(per_class: dict, work, peaks: dict) -> dict:
+    """Per family: device ms per step (summed over its launches), algorithmic bytes and flops per step, the
+    bound (tensor when flops / sustained bf16 exceed bytes / HBM) and the achieved rate against that peak."""
+    bw, tf = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops_sustained"] * 1e12
+    out = {}
+    for fam, classes in FAMILIES.items():
+        ms = sum(per_class.get(k, (0.0, 0))[0] for k in classes)
+        n = sum(per_class.get(k, (0.0, 0))[1] for k in classes)
+        by = sum(cnt * b for kc, cnt, b, f in work if kc in classes)
+        fl = sum(cnt * f for kc, cnt, b, f in work if kc in classes)
+        if ms <= 0 or n == 0:
+            continue
+        tensor = fl / tf > by / bw
+        ach = fl / (ms / 1e3) / 1e12 if tensor else by / (ms / 1e3) / 1e9
+        peak = peaks["bf16_tflops_sustained"] if tensor else peaks["hbm_gbs"]
+        out[fam] = {"bound": "tensor" if tensor else "hbm", "achieved": round(ach, 1), "peak": peak,
+                    "unit": "TFLOP/s" if tensor else "GB/s", "frac": round(ach / peak, 4), "ms_per_step": round(ms, 4),
+                    "launches": n, "algorithmic_gb": round(by / 1e9, 4), "algorithmic_tflop": round(fl / 1e12, 4)}
+    return out
+
+
 def source_digest(kclass: str) -> str:
     """Digest of the sources that build a kernel class (recorded traffic is used only while it matches)."""
     shared = ["common.cuh", "launch.h"]
@@ -278,27 +327,58 @@ def blas_threads():
     return os.cpu_count()
 
 
-def run_reference(args):
-    """The oracle on the host cores: each step is one request of the workload (requests cycle)."""
-    case = make_workload(args, fs.SEEDS.get(args.workload, 1234), "cpu")
-    model64 = {k: ([t.to(torch.float64).numpy() for t in v] if isinstance(v, list) else v.to(torch.float64).numpy())
-               for k, v in case.model.items()}
+def oracle_model(model: dict, share: float = 0.5):
+    """The weights as float64 arrays (an input form the oracle takes as is) when they fit in `share` of the
+    host's free memory, else as given (the oracle then converts the layers it reads on every call).
+    Returns (model, converted)."""
+    import psutil
+    tensors = [t for v in model.values() for t in (v if isinstance(v, list) else [v])]
+    if sum(t.numel() for t in tensors) * 8 > share * psutil.virtual_memory().available:
+        return model, False
+    f64 = lambda t: t.detach().cpu().to(torch.float64).numpy()
+    return {k: ([f64(t) for t in v] if isinstance(v, list) else f64(v)) for k, v in model.items()}, True
+
+
+def cpu_oracle_sample(case: fs.Case, model, seconds: float, max_requests=None):
+    """Time the oracle one request per call, in request order, until `seconds` of CPU work have run (at
+    least one request).  Returns (decoded tokens, seconds, requests run)."""
     N = case.work.n_requests
+    limit = N if max_requests is None else min(N, max_requests)
+    tok, secs, n = 0, 0.0, 0
+    while n < limit and (secs < seconds or n == 0):
+        t, dt = oracle_tokens_per_s(case, [n], model)
+        tok, secs, n = tok + t, secs + dt, n + 1
+    return tok, secs, n
+
+
+def run_reference(args):
+    """The oracle on the host cores: each step is one request of the workload (requests cycle).  Only the
+    requests the run visits are generated (same shapes, distributions and seed), so that the 8B shape's
+    page pool fits on the host; the weights are converted to float64 once, before the timed steps, when
+    the host has room for them."""
+    shape, work, base = resolve_workload(args.workload)
+    n_used = max(1, min(work.n_requests if args.requests is None else args.requests, args.warmup + args.steps))
+    case = make_workload(args, base, "cpu", requests=n_used)
+    full = fs.Case(case.shape, dataclasses.replace(case.work, n_requests=work.n_requests if args.requests is None
+                                                   else args.requests), None, None, case.seed)
+    model, converted = oracle_model(case.model)
     for i in range(args.warmup):
-        oracle_tokens_per_s(case, [i % N], model64)
+        oracle_tokens_per_s(case, [i % n_used], model)
     tok, secs = 0, 0.0
     for i in range(args.steps):
-        t, dt = oracle_tokens_per_s(case, [(args.warmup + i) % N], model64)
+        t, dt = oracle_tokens_per_s(case, [(args.warmup + i) % n_used], model)
         tok += t
         secs += dt
     value = tok / secs if secs > 0 else 0.0
     cores = blas_threads()
-    sample = (f"one of {N} requests per step (cycling), float64 oracle, weights converted to float64 once "
-              f"before the timed steps")
+    sample = (f"one request per step, cycling over the first {n_used} requests of the workload (same shapes "
+              f"and distributions), float64 oracle, " +
+              ("weights converted to float64 once before the timed steps" if converted else
+               "weights converted inside every step (host memory too small to hold them in float64)"))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "desc": workload_desc(case), "parallelism": "host cores"},
+            "config": {"workload": args.workload, "desc": workload_desc(full), "parallelism": "host cores"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -583,21 +663,29 @@ def main():
                          "kept_rows": R})
 
     # ---- the whole step against its roofline (sum over launches of the slower of bytes and flops)
-    step_roof = step_roofline(step_work(case, R, kept.tolist(), plen.tolist()), peaks, max_ms / K)
+    work_list = step_work(case, R, kept.tolist(), plen.tolist())
+    step_roof = step_roofline(work_list, peaks, max_ms / K)
     step_roof["peak_source"] = f"{peak_src} (HBM copy; sustained bf16)"
+    families = family_rooflines(per_class, work_list, peaks) if per_class else None
+    weights_gb = sum(t.numel() * t.element_size() for v in case.model.values()
+                     for t in (v if isinstance(v, list) else [v])) / 1e9
+    kv_gb = float(plen.sum()) * shp.n_layers * 2 * shp.n_kv_heads * shp.head_dim * case.batch["kv_pool"].element_size() / 1e9
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        host = fs.Case(shp, w, {k: ([x.cpu() for x in v] if isinstance(v, list) else v.cpu())
-                                for k, v in case.model.items()},
-                       {k: v.cpu() for k, v in case.batch.items()}, case.seed)
-        host.batch["block_tokens"], host.batch["mask"], host.batch["ibc"] = tok0.cpu(), mask0.cpu(), ibc0.cpu()
+        # the oracle reads the model and the batch from host copies, and the page pool (tens of GB at the 8B
+        # shape) page by page from the device
         del st
-        nreq = min(N, args.cpu_baseline_requests)
-        ctok, csec = oracle_tokens_per_s(host, range(nreq))
+        host_batch = {k: (v if k == "kv_pool" else v.cpu()) for k, v in case.batch.items()}
+        host_batch["block_tokens"], host_batch["mask"], host_batch["ibc"] = tok0.cpu(), mask0.cpu(), ibc0.cpu()
+        host = fs.Case(shp, w, None, host_batch, case.seed)
+        model64, converted = oracle_model(case.model)
+        ctok, csec, nreq = cpu_oracle_sample(host, model64, 20.0, args.cpu_baseline_requests)
         cpu = {"value": ctok / csec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{nreq} of {N} requests of the same batch, one oracle call ({csec:.1f} s, "
-                         f"float64, weight conversion included)"}
+               "sample": f"{nreq} of {N} requests of the same batch, one oracle call each ({csec:.1f} s of "
+                         f"float64 work; weights converted to float64 " +
+                         ("once, untimed)" if converted else "inside every call)")}
+        del model64
 
     if rank == 0:
         line = {
@@ -611,10 +699,12 @@ def main():
                        "decoded_per_step": total_decoded / K / world,
                        "launch": "eager focus_step calls" if args.eager else
                                  "CUDA graph of one focus_step, one replay per step (tokens/mask restored by two copies)",
-                       "l2": "inputs larger than L2 (3.4 GB of weights and ~2.4 GB of KV pages streamed per step)",
+                       "l2": f"inputs larger than L2 ({weights_gb:.1f} GB of weights and {kv_gb:.1f} GB of prefix KV "
+                             f"pages read per step, against a 126 MB L2)",
                        "parallelism": f"replicas x{world} (requests sharded, no collective)"},
             "gpu_launches": launches_per_step * K,
-            "clocks": clocks, "roofline": roofline, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clocks, "roofline": roofline, "step_roofline": step_roof, "families": families,
+            "cpu_baseline": cpu, "e2e": e2e,
             "per_class_ms_per_step": {k: round(v[0], 4) for k, v in per_class.items()} if per_class else None,
         }
         print(json.dumps(line), flush=True)

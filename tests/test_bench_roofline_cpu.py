@@ -78,3 +78,28 @@ def test_step_roofline_of_the_bench_workload_is_dominated_by_streams():
     weights = s.n_layers * (s.hidden * (s.n_q_heads + 2 * s.n_kv_heads) * s.head_dim + s.n_q_heads * s.head_dim * s.hidden
                             + 3 * s.hidden * s.ffn) * 2 + s.vocab * s.hidden * 2
     assert r["algorithmic_gb"] * 1e9 > weights  # every weight is read at least once per step
+
+
+def test_families_sum_their_kernel_classes_and_take_the_slower_bound():
+    # the 8B shape with 14 kept rows per request: the kept-row GEMMs are one tensor-bound family, the ragged
+    # attention an HBM-bound one
+    case = _case("sdar8b_n256_b64")
+    N = case.work.n_requests
+    work = bench.step_work(case, R=14 * N, kept_per_req=[14] * N, plen=[1280] * N)
+    per_class = {kc: (2.0, 34) for kc, _, _, _ in work}
+    peaks = {"hbm_gbs": 6541.8, "bf16_tflops_sustained": 1365.2}
+    fam = bench.family_rooflines(per_class, work, peaks)
+    kept = fam["gemm_kept_rows"]
+    assert kept["ms_per_step"] == 8.0 and kept["launches"] == 4 * 34 and kept["bound"] == "tensor"
+    fl = sum(n * f for kc, n, _, f in work if kc in ("gemm_qkv", "gemm_o", "gemm_gateup", "gemm_down"))
+    assert abs(kept["algorithmic_tflop"] - fl / 1e12) < 1e-3
+    assert abs(kept["achieved"] - fl / 8e-3 / 1e12) < 0.1
+    assert fam["attention_ragged"]["bound"] == "hbm" and fam["attention_ragged"]["unit"] == "GB/s"
+
+
+def test_sweep_workload_names_resolve_to_the_sweep_recipe():
+    shape, work, seed = bench.resolve_workload("sweep_n256_b64_f1.0")
+    assert shape == fs.MODEL_SHAPES["sdar1.7b"] and seed == fs.SEEDS["sweep"]
+    assert (work.n_requests, work.block, work.forced_keep_frac, work.prefix) == (256, 64, 1.0, ("uniform", 256, 4096))
+    shape, work, seed = bench.resolve_workload("sdar8b_n256_b64")
+    assert shape == fs.MODEL_SHAPES["sdar8b"] and work.n_requests == 256 and seed == fs.SEEDS["sdar8b_n256_b64"]
