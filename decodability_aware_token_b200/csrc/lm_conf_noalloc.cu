@@ -25,7 +25,7 @@ using namespace tc;
 
 // maximum sizes served by the fixed scratch array
 constexpr int kNaRows = 256;                    // hidden rows per call
-constexpr int kNaDim = 4096;                    // hidden size (a multiple of 64)
+constexpr int kNaDim = 4096;                    // hidden size (a multiple of 128)
 constexpr int kNaVocab = 163840;                // vocabulary size
 constexpr int kNaBN = 128;                      // vocabulary columns per statistics tile
 constexpr int kNaTiles = kNaVocab / kNaBN;      // 1280 tiles
@@ -122,6 +122,12 @@ extern "C" int focus_lm_head_conf_noalloc(const float* hidden, int32_t rows, int
                                           float* conf, int32_t* top_id, void* stream) {
     if (!hidden || !final_norm || !lm_head || !conf || !top_id || rows < 0 || hidden_dim <= 0 || vocab <= 0 ||
         !(rms_eps >= 0.f))
+        return FOCUS_ERR_INVALID_ARG;
+    // the kernels read hidden rows as float4, final_norm four bf16 at a time, and lm_head through a TMA tensor
+    // map (16-byte base); outputs are written per element
+    if (reinterpret_cast<uintptr_t>(hidden) % 16 || reinterpret_cast<uintptr_t>(final_norm) % 8 ||
+        reinterpret_cast<uintptr_t>(lm_head) % 16 || reinterpret_cast<uintptr_t>(conf) % 4 ||
+        reinterpret_cast<uintptr_t>(top_id) % 4)
         return FOCUS_ERR_INVALID_ARG;
     if (rows > kNaRows || hidden_dim > kNaDim || vocab > kNaVocab) return FOCUS_ERR_LIMITS;
     if (hidden_dim % 128) return FOCUS_ERR_UNSUPPORTED;

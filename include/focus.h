@@ -279,18 +279,22 @@ int focus_profile_end(focus_ctx* ctx, float* total_ms, int32_t* launches);
  * allocator (a thread recording a CUDA graph, a serving loop with a fixed memory budget, a plug-in
  * whose host framework owns all device memory).  It runs the step's last stage -- final RMSNorm,
  * LM head, max-softmax confidence, top id (lowest id among equal maxima) -- on hidden rows the
- * caller holds, with the same kernels and arithmetic as focus_step, and allocates nothing: its
- * intermediate data lives in one fixed array of about 5.75 MiB inside the library, which every GPU
- * that loads the library keeps until the process exits.
+ * caller holds, and allocates nothing: its intermediate data lives in one fixed array of about
+ * 5.75 MiB inside the library, which every GPU that loads the library keeps until the process exits.
+ * It uses focus_step's norm routine and LM-head GEMM kernel; top ids equal focus_step's, confidences
+ * equal them up to the float summation order in which the vocabulary tiles are merged.
  *
- *   hidden      [rows, hidden_dim] float32, device: residual-stream rows (e.g. focus_step_out.hidden)
- *   final_norm  [hidden_dim] bf16, device;  lm_head [vocab, hidden_dim] bf16, device
- *   conf        [rows] float32, device (out); top_id [rows] int32, device (out)
+ *   hidden      [rows, hidden_dim] float32, device, 16-byte aligned: residual-stream rows (e.g.
+ *               focus_step_out.hidden)
+ *   final_norm  [hidden_dim] bf16, device, 8-byte aligned;  lm_head [vocab, hidden_dim] bf16, device,
+ *               16-byte aligned
+ *   conf        [rows] float32, device (out); top_id [rows] int32, device (out); both 4-byte aligned
  *   stream      cudaStream_t (NULL = legacy default stream); the call is asynchronous
  *
  * Limits: rows <= 256, hidden_dim <= 4096 and a multiple of 128, vocab <= 163840; larger sizes return
  * FOCUS_ERR_LIMITS (FOCUS_ERR_UNSUPPORTED for a hidden_dim that is not a multiple of 128) and launch
- * nothing.  rows == 0 returns FOCUS_OK at once.  The first call on a device looks up the array's
+ * nothing; a misaligned pointer returns FOCUS_ERR_INVALID_ARG before any device call.  rows == 0
+ * returns FOCUS_OK at once.  The first call on a device looks up the array's
  * device address (with that device current) and must therefore come before any stream capture on
  * that device.  All calls on a device share the array: calls that may overlap on the GPU race on it
  * and must be serialised by the caller.  If a bounded wait inside the GEMM expires, conf is NaN and

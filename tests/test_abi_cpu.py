@@ -121,6 +121,18 @@ def test_lm_head_noalloc_checks_before_the_device(rows, dim, vocab, eps, code):
     assert lib.focus_lm_head_conf_noalloc(_P, rows, dim, _P, _P, vocab, eps, _P, _P, None) == code
 
 
+@pytest.mark.parametrize("which,offset", [(0, 8), (0, 4), (1, 2), (2, 8), (3, 2), (4, 1)])
+def test_lm_head_noalloc_rejects_misaligned_buffers(which, offset):
+    """hidden 16-byte, final_norm 8-byte, lm_head 16-byte, conf / top_id 4-byte aligned (a torch view with an
+    element offset would otherwise fault on the device); refused before any device call."""
+    lib = _abi.load()
+    ptrs = [C.c_void_p(4096) for _ in range(5)]
+    ptrs[which] = C.c_void_p(4096 + offset)
+    h, nrm, w, conf, top = ptrs
+    assert lib.focus_lm_head_conf_noalloc(h, 4, 2048, nrm, w, 1000, 1e-6, conf, top, None) == \
+        _abi.FOCUS_ERR_INVALID_ARG
+
+
 def test_lm_head_noalloc_rejects_null_buffers():
     lib = _abi.load()
     for i in range(5):

@@ -5,7 +5,8 @@ CUDA graph, a fixed-budget serving loop, a plug-in inside a framework that owns 
 It keeps its intermediate data in a fixed array inside the library, shared by every call.  This test
 calls it through the C ABI twice in a row -- all kept rows, then a shorter prefix of them, so stale
 contents of the shared array would show -- and checks both results against the conf / top id that
-focus_step computed for the same rows.  This file is collected last on purpose.
+focus_step computed for the same rows, and the first one also against the float64 oracle's final norm,
+LM head and max-softmax on those rows.  This file is collected last on purpose.
 """
 import ctypes as C
 
@@ -45,6 +46,7 @@ def test_lm_head_conf_without_allocation_matches_focus_step():
     top = torch.full((R,), -7, dtype=torch.int32, device=dev)
     stream = C.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     frac = 2e-2   # the bf16 tolerance of the parity tests: max-abs <= frac x RMS
+    first = None
     for rows in (R, max(1, R // 2)):
         conf.fill_(-1.0)
         top.fill_(-7)
@@ -58,6 +60,23 @@ def test_lm_head_conf_without_allocation_matches_focus_step():
         assert np.abs(got_c[:rows] - want).max() <= frac * np.sqrt(np.mean(want ** 2))
         np.testing.assert_array_equal(got_t[:rows], ref_top[:rows])
         assert np.all(got_c[rows:] == -1.0) and np.all(got_t[rows:] == -7)   # nothing written past `rows`
+        if first is None:
+            first = (got_c.copy(), got_t.copy())
+
+    # the first call against the oracle (float64 norm, logits, max-softmax, lowest id among the maxima):
+    # confidences within 2e-2 x RMS, top ids equal wherever the oracle's top-1 margin exceeds the logit
+    # error that tolerance allows (2e-2 x sqrt(D) x RMS of the LM-head weights), else within it
+    from oracle import focus_oracle as fo
+    h64 = hidden.cpu().double().numpy()
+    g64, w64 = fo._f64(case.model["final_norm"]), fo._f64(case.model["lm_head"])
+    c64, t64, _, margin = fo.lm_head_conf(h64, g64, w64, shp.rms_eps)
+    got_c, got_t = first
+    assert np.abs(got_c - c64).max() <= frac * np.sqrt(np.mean(c64 ** 2))
+    gate = frac * np.sqrt(shp.hidden) * float(np.sqrt(np.mean(w64 ** 2)))
+    z = fo.rms_norm(h64, g64, shp.rms_eps) @ w64.T
+    for r in range(R):
+        if got_t[r] != t64[r]:
+            assert margin[r] <= gate and z[r, t64[r]] - z[r, got_t[r]] <= gate, (r, got_t[r], t64[r], margin[r])
 
     # sizes beyond the fixed array are refused before anything is launched
     rc = lib.focus_lm_head_conf_noalloc(_p(hidden), 257, shp.hidden, _p(model["final_norm"]), _p(model["lm_head"]),
