@@ -15,11 +15,16 @@ each iteration runs at most two calls on contiguous slot ranges -- the focused s
 steps (first steps and refreshes) -- and then commits the blocks whose refresh just ran.  Finished
 requests leave their slot at once and waiting ones take it (continuous batching).
 
-Admission (the effective batch): a request in a focused step costs at most k_max rows in layers
-2..L-1, one in a dense step costs B.  A waiting request is admitted while a slot is free, the pages for
-all its blocks can be reserved, and the summed cost of the active requests plus B (its dense first step)
-stays within ``row_budget``.  A dense engine spending N x B rows per step admits N requests; with the
-same budget, focused requests cost k_max, so up to N x B / k_max of them run at once.
+The row budget (the effective batch): a request in a focused step costs at most k_max rows in layers
+2..L-1, one in a dense step costs B, and no iteration runs more than ``row_budget`` rows.  A waiting
+request is admitted while a slot is free, the pages for all its blocks can be reserved, and the summed
+cost of the active requests plus B (its dense first step) stays within the budget.  Every iteration then
+runs all focused steps and as many dense steps (first steps and refreshes, oldest admission first) as
+still fit; the other dense steps wait for a later iteration.  The focused steps always fit (each
+admission kept every active request's cost, at least k_max, within the budget), and when no request is
+focused at least one dense step runs, so every request keeps moving.  A dense engine spending N x B rows
+per step admits N requests; with the same budget, focused requests cost k_max, so up to N x B / k_max of
+them run at once.
 
 Readings (the pages describe no scheduler): first come, first served among arrived requests; a
 request's prompt pages and the pages allocated for its blocks return to the pool when it finishes
@@ -66,9 +71,10 @@ class IterationStats:
     iteration: int
     active: int                   # requests in slots during the iteration
     focused: int                  # of which in a focused step
-    dense: int                    # of which in a dense step (first step or refresh)
-    row_cost: int                 # focused * k_max + dense * B
+    dense: int                    # of which ran a dense step (first step or refresh)
+    row_cost: int                 # focused * k_max + dense * B: rows run, at most row_budget
     committed: int                # blocks committed at the end of the iteration
+    deferred: int = 0             # requests whose dense step waits for a later iteration (budget full)
 
 
 class FocusEngine:
@@ -223,6 +229,14 @@ class EffectiveBatchScheduler:
                 return lo
             self._swap(lo, hi)
 
+    def _order_dense(self, start: int) -> None:
+        """Sort the dense slots [start, n) by admission (oldest first), so the ones that fit come first."""
+        n = len(self.slot_req)
+        key = lambda i: (self.slot_req[i]["admitted"], self.slot_req[i]["req"].rid)
+        for i in range(start, n):  # selection sort through slot swaps (a handful of slots)
+            j = min(range(i, n), key=key)
+            self._swap(i, j)
+
     def _view(self, a: int, b: int) -> Dict[str, torch.Tensor]:
         return {"block_tokens": self.tokens[a:b], "mask": self.mask[a:b], "prefix_len": self.prefix_len[a:b],
                 "page_table": self.page_table[a:b], "kv_pool": self.kv_pool, "ibc": self.ibc[a:b]}
@@ -235,9 +249,12 @@ class EffectiveBatchScheduler:
         """Admit, run the focused and the dense steps, move every request to its next phase, commit the
         blocks whose refresh ran, retire finished requests."""
         self._admit()
-        n = len(self.slot_req)
+        n_active = len(self.slot_req)
         n_f = self._partition()
-        cost = sum(self._cost(r) for r in self.slot_req)
+        self._order_dense(n_f)
+        fit = (self.row_budget - n_f * self.k_max) // self.B
+        n = n_f + max(0, min(n_active - n_f, fit))     # slots [0, n) run; dense slots beyond wait
+        cost = n_f * self.k_max + (n - n_f) * self.B
         if n_f > 0:
             self.engine.step(self._view(0, n_f), dense=False)
         if n > n_f:
@@ -245,7 +262,7 @@ class EffectiveBatchScheduler:
         masked = self.mask[:n].to("cpu").bool().any(dim=1).tolist() if n else []
         committed = 0
         finished = []
-        for i, rec in enumerate(self.slot_req):
+        for i, rec in enumerate(self.slot_req[:n]):
             rec["block_steps"] += 1 if rec["phase"] != _DENSE_REFRESH else 0
             if rec["phase"] == _DENSE_REFRESH:
                 self.engine.commit(self._view(i, i + 1))
@@ -274,7 +291,7 @@ class EffectiveBatchScheduler:
             if not self.keep_pages:
                 self.free.extend(rec["pages"])
             self.free.extend(rec["reserved"])  # none left once every block is placed
-        st = IterationStats(self.iteration, n, n_f, n - n_f, cost, committed)
+        st = IterationStats(self.iteration, n_active, n_f, n - n_f, cost, committed, n_active - n)
         self.stats.append(st)
         self.iteration += 1
         return st
