@@ -6,8 +6,10 @@
 //   EPI_QKV:     rotary embedding of the query / key heads, queries to q, keys and values to the cache
 //
 // GEMMs of at most 256 rows (the kept rows and the LM head) run on the swapped kernel (features on the
-// MMA's M side, tokens on N, split K over a thread-block cluster); the full-block GEMMs of layers 0-1 on
-// the row-major kernel.
+// MMA's M side, tokens on N, split K over a thread-block cluster).  GEMMs with more rows (the full-block
+// GEMMs of layers 0-1, the kept rows of large batches) run on the persistent kernel (tc_gemm_persist.cuh:
+// one CTA per SM, 128 x 256 or 128 x 128 tiles, two TMEM accumulators so that epilogues overlap the next
+// tile's MMAs) when they have enough tiles to fill the SMs, else on the one-tile-per-CTA row-major kernel.
 //
 // One CTA computes a (128 * MSUB) x BN tile (MSUB accumulators of 128 x BN fp32 in TMEM) over a range of
 // 64-wide K blocks.  Warp roles: warp 0 lane 0 issues TMA loads into a STAGES-deep shared-memory ring,
@@ -22,6 +24,7 @@
 
 #include "tc_gemm.h"
 #include "tc_gemm_kernel.cuh"
+#include "tc_gemm_persist.cuh"
 
 namespace focus {
 
@@ -37,6 +40,7 @@ using namespace tc;
 // all rows beyond the live row count exit after the wait.
 constexpr int kBN = 128, kStages = 4;
 constexpr int kSmallRows = 256;  // GEMMs with at most this many rows run on the swapped kernel
+constexpr bool kUsePairs = false;  // many-row GEMMs on CTA pairs (tc_gemmp2_kernel) where they fill the GPU
 using Big = TcShape<kBN, 2, kStages>;
 using Small = TcShape<kBN, 1, kStages>;
 
@@ -50,9 +54,11 @@ struct TcPlan {
     CUtensorMap map_h1, map_o1, map_act1;     // 128-row boxes
     CUtensorMap map_h32, map_o32, map_act32;  // 32-row boxes: token operand of the swapped kernel
     std::unordered_map<const void*, CUtensorMap> wmap;   // weight pointer -> map (box rows = tile N or N/2)
+    std::unordered_map<const void*, CUtensorMap> wmap2;  // the same with 256-row boxes (128 for gate / up)
     int* err;
     int sms;
     int max_clusters[kTMaxSplits + 1];  // co-resident clusters of the swapped kernel with s CTAs (0: not launchable)
+    int max_pairs;                      // co-resident CTA pairs of the paired persistent kernel (0: not used)
 };
 
 
@@ -90,10 +96,22 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
         p->wmap[w.wup[l]] = m;
         ok = ok && make_map(&m, w.wdown[l], dm.D, dm.F, kBN);
         p->wmap[w.wdown[l]] = m;
+        ok = ok && make_map(&m, w.wqkv[l], dm.qkv, dm.D, 2 * kBN);
+        p->wmap2[w.wqkv[l]] = m;
+        ok = ok && make_map(&m, w.wo[l], dm.D, HD, 2 * kBN);
+        p->wmap2[w.wo[l]] = m;
+        ok = ok && make_map(&m, w.wgate[l], dm.F, dm.D, kBN);
+        p->wmap2[w.wgate[l]] = m;
+        ok = ok && make_map(&m, w.wup[l], dm.F, dm.D, kBN);
+        p->wmap2[w.wup[l]] = m;
+        ok = ok && make_map(&m, w.wdown[l], dm.D, dm.F, 2 * kBN);
+        p->wmap2[w.wdown[l]] = m;
     }
     CUtensorMap m;
     ok = ok && make_map(&m, w.lm_head, dm.V, dm.D, kBN);
     p->wmap[w.lm_head] = m;
+    ok = ok && make_map(&m, w.lm_head, dm.V, dm.D, 2 * kBN);
+    p->wmap2[w.lm_head] = m;
     if (!ok) {
         delete p;
         return FOCUS_ERR_CUDA;
@@ -111,7 +129,19 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
          set_smem((const void*)tc_gemmt_kernel<EPI_RESID>, kTSmem) &&
          set_smem((const void*)tc_gemmt_kernel<EPI_QKV>, kTSmem) &&
          set_smem((const void*)tc_gemmt_kernel<EPI_SWIGLU>, kTSmem) &&
-         set_smem((const void*)tc_gemmt_kernel<EPI_LMHEAD>, kTSmem);
+         set_smem((const void*)tc_gemmt_kernel<EPI_LMHEAD>, kTSmem) &&
+         set_smem((const void*)tc_gemmp_kernel<256, EPI_SWIGLU>, PShape<256>::SMEM) &&
+         set_smem((const void*)tc_gemmp_kernel<256, EPI_LMHEAD>, PShape<256>::SMEM) &&
+         set_smem((const void*)tc_gemmp_kernel<256, EPI_RESID>, PShape<256>::SMEM) &&
+         set_smem((const void*)tc_gemmp_kernel<256, EPI_QKV>, PShape<256>::SMEM) &&
+         set_smem((const void*)tc_gemmp_kernel<128, EPI_SWIGLU>, PShape<128>::SMEM) &&
+         set_smem((const void*)tc_gemmp_kernel<128, EPI_LMHEAD>, PShape<128>::SMEM) &&
+         set_smem((const void*)tc_gemmp_kernel<128, EPI_RESID>, PShape<128>::SMEM) &&
+         set_smem((const void*)tc_gemmp_kernel<128, EPI_QKV>, PShape<128>::SMEM) &&
+         set_smem((const void*)tc_gemmp2_kernel<EPI_SWIGLU>, kP2Smem) &&
+         set_smem((const void*)tc_gemmp2_kernel<EPI_LMHEAD>, kP2Smem) &&
+         set_smem((const void*)tc_gemmp2_kernel<EPI_RESID>, kP2Smem) &&
+         set_smem((const void*)tc_gemmp2_kernel<EPI_QKV>, kP2Smem);
     int dev = 0;
     p->sms = 0;
     ok = ok && cudaGetDevice(&dev) == cudaSuccess &&
@@ -139,6 +169,26 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
         p->max_clusters[cs] = n;
     }
     ok = ok && p->max_clusters[1] > 0;
+    p->max_pairs = 0;
+    if (ok && kUsePairs) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(2, 1, 1);
+        cfg.blockDim = dim3(192, 1, 1);
+        cfg.dynamicSmemBytes = kP2Smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, tc_gemmp2_kernel<EPI_RESID>, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            n = 0;
+        }
+        p->max_pairs = n;
+    }
     if (!ok) {
         delete p;
         return FOCUS_ERR_CUDA;
@@ -186,6 +236,63 @@ int tc_gemm_swapped(TcPlan* p, Epi epi, GemmArgs g, cudaStream_t s) {
     return e == cudaSuccess ? 1 : -1;
 }
 
+// Persistent kernel for many rows: 128 x bn tiles over min(SMs, tiles) CTAs.
+template <int BN>
+int tc_gemm_persistent(TcPlan* p, Epi epi, GemmArgs g, int tiles, cudaStream_t s) {
+    const CUtensorMap* a = g.A == p->h ? &p->map_h1 : g.A == p->o ? &p->map_o1 : &p->map_act1;
+    auto& wm = BN == 256 ? p->wmap2 : p->wmap;
+    const CUtensorMap* b = &wm.find(g.B)->second;
+    const CUtensorMap* b2 = epi == EPI_SWIGLU ? &wm.find(g.B2)->second : b;
+    if (epi == EPI_LMHEAD) {
+        g.n_tiles = (g.N + kBN - 1) / kBN;  // statistics per 128 vocabulary columns, as the combine reads them
+        g.tile_n = kBN;
+    }
+    const dim3 grid(tiles < p->sms ? tiles : p->sms, 1, 1), blk(192);
+    const int smem = PShape<BN>::SMEM;
+    switch (epi) {
+        case EPI_SWIGLU: return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_SWIGLU>, grid, blk, smem, s, 0, *a, *b, *b2, g, p->err));
+        case EPI_LMHEAD: return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_LMHEAD>, grid, blk, smem, s, 0, *a, *b, *b2, g, p->err));
+        case EPI_RESID: return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_RESID>, grid, blk, smem, s, 0, *a, *b, *b2, g, p->err));
+        case EPI_QKV: return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_QKV>, grid, blk, smem, s, 0, *a, *b, *b2, g, p->err));
+        default: return -1;
+    }
+}
+
+// Paired persistent kernel: 256 x 256 tiles over min(co-resident pairs, tiles) clusters of 2 CTAs.
+int tc_gemm_pairs(TcPlan* p, Epi epi, GemmArgs g, int tiles, cudaStream_t s) {
+    const CUtensorMap* a = g.A == p->h ? &p->map_h1 : g.A == p->o ? &p->map_o1 : &p->map_act1;
+    // 128-row weight boxes: each rank loads half of the tile's 256 weight rows (gate or up for SwiGLU)
+    const CUtensorMap* b = &p->wmap2.find(g.B)->second;
+    const CUtensorMap* b2 = b;
+    if (epi == EPI_SWIGLU) {
+        b = &p->wmap2.find(g.B)->second;
+        b2 = &p->wmap2.find(g.B2)->second;
+    } else {
+        b = &p->wmap.find(g.B)->second;
+        b2 = b;
+    }
+    if (epi == EPI_LMHEAD) {
+        g.n_tiles = (g.N + kBN - 1) / kBN;
+        g.tile_n = kBN;
+    }
+    const int pairs = tiles < p->max_pairs ? tiles : p->max_pairs;
+    const dim3 grid(2 * pairs, 1, 1), blk(192);
+    switch (epi) {
+        case EPI_SWIGLU: return launched(launch_pdl(tc_gemmp2_kernel<EPI_SWIGLU>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, g, p->err));
+        case EPI_LMHEAD: return launched(launch_pdl(tc_gemmp2_kernel<EPI_LMHEAD>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, g, p->err));
+        case EPI_RESID: return launched(launch_pdl(tc_gemmp2_kernel<EPI_RESID>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, g, p->err));
+        case EPI_QKV: return launched(launch_pdl(tc_gemmp2_kernel<EPI_QKV>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, g, p->err));
+        default: return -1;
+    }
+}
+
+// Column tiles of width bn (0 if the epilogue needs whole tiles and N does not divide).
+int persist_col_tiles(Epi epi, int N, int bn) {
+    if (epi == EPI_SWIGLU) return N % (bn / 2) ? 0 : N / (bn / 2);
+    if (epi == EPI_LMHEAD) return (N + bn - 1) / bn;  // a partial last tile is masked column by column
+    return N % bn ? 0 : N / bn;
+}
+
 }  // namespace
 
 int tc_gemm(TcPlan* p, Epi epi, const GemmArgs& g0, cudaStream_t s) {
@@ -193,6 +300,25 @@ int tc_gemm(TcPlan* p, Epi epi, const GemmArgs& g0, cudaStream_t s) {
     if (epi == EPI_PARTIAL) return -1;  // partial sums are the CUDA-core path's; these kernels fuse their epilogues
     GemmArgs g = g0;
     if (g.M_bound <= kSmallRows) return tc_gemm_swapped(p, epi, g, s);
+    {
+        // Persistent kernel when there are enough tiles to fill the SMs.  Of 256- and 128-wide tiles take the
+        // one with the shorter expected time: full waves of tiles (at the row bound) x tile width, a 128-wide
+        // tile costing 15 % more per column (half-width MMAs, twice the A traffic per flop).
+        const int mt = (g.M_bound + 127) / 128;
+        const int n256 = persist_col_tiles(epi, g.N, 256), n128 = persist_col_tiles(epi, g.N, 128);
+        const long long t256 = (long long)mt * n256, t128 = (long long)mt * n128;
+        const double c256 = n256 ? (double)((t256 + p->sms - 1) / p->sms) * 256.0 : 1e30;
+        const double c128 = n128 ? (double)((t128 + p->sms - 1) / p->sms) * 128.0 * 1.15 : 1e30;
+        if (p->max_pairs > 0 && n256) {
+            // pairs: 256 x 256 tiles, one round = max_pairs tiles; a round takes about as long as a round of
+            // 128 x 256 tiles on single CTAs, at two thirds of their operand bytes per flop
+            const long long tp = (long long)((g.M_bound + 255) / 256) * n256;
+            const double cp = (double)((tp + p->max_pairs - 1) / p->max_pairs) * 256.0 * (2.0 * p->max_pairs / p->sms);
+            if (tp >= p->max_pairs && cp <= c256 && cp <= c128) return tc_gemm_pairs(p, epi, g, (int)tp, s);
+        }
+        if (n256 && t256 >= p->sms && c256 <= c128) return tc_gemm_persistent<256>(p, epi, g, (int)t256, s);
+        if (n128 && t128 >= p->sms) return tc_gemm_persistent<128>(p, epi, g, (int)t128, s);
+    }
     // residual and QKV GEMMs whose 256-row tiles would leave SMs idle take 128-row tiles
     const int n_tiles_big = (g.N + kBN - 1) / kBN;
     const bool rows128 = (epi == EPI_RESID || epi == EPI_QKV) &&
