@@ -59,9 +59,10 @@ def parse():
     ap.add_argument("--eager", action="store_true", help="time eager focus_step calls instead of graph replays")
     ap.add_argument("--layers", type=int, default=None, help="override the layer count (profiling cases)")
     ap.add_argument("--requests", type=int, default=None, help="override the request count (profiling cases)")
-    ap.add_argument("--mode", choices=["step", "block"], default="step",
+    ap.add_argument("--mode", choices=["step", "block", "schedule"], default="step",
                     help="step: one focused step (the default measurement); block: whole blocks decoded to "
-                         "completion and committed (dense first step, focused steps, dense refresh, commit)")
+                         "completion and committed (dense first step, focused steps, dense refresh, commit); "
+                         "schedule: a trace of requests through the effective-batch scheduler, focused vs dense")
     return ap.parse_args()
 
 
@@ -189,7 +190,8 @@ def algorithmic_work(kclass: str, case: fs.Case, R: int, kept_per_req, plen, spl
 def step_work(case: fs.Case, R: int, kept_per_req, plen):
     """Every launch of one step as (kernel class, launches, algorithmic bytes, flops per launch), in the
     step's order: embedding + norm; layers 0-1 on all N*B rows (QKV, attention with importance, O,
-    norm, gate/up, down, and a norm between the layers); selection; the norm that gathers the kept rows;
+    norm, gate/up, down, and a norm between the layers); selection and the row map; the norm that gathers
+    the kept rows;
     layers 2..L-1 on the R kept rows (QKV, ragged attention, O, norm, gate/up, down, norm); LM head;
     combine + decode.  Norms read the float32 residual and write bf16 rows (the gathering norm also
     writes the compacted float32 rows)."""
@@ -205,7 +207,10 @@ def step_work(case: fs.Case, R: int, kept_per_req, plen):
         by, fl = algorithmic_work(kc, case, R, kept_per_req, plen)
         work.append((kc, n, by, fl))
     work.append(("row_norm", 3, rows_full * D * (4 + e), 0.0))
-    work.append(("select", 1, 2 * N * s.n_kv_heads * B * 4 + 2 * N * B, 0.0))
+    # the importance partials (per KV head and 64-vector query tile) and the mask, then the row map
+    q_tiles = -(-(B * (s.n_q_heads // s.n_kv_heads)) // 64) if s.dtype == "bf16" else 1
+    work.append(("select", 1, 2 * N * s.n_kv_heads * q_tiles * B * 4 + N * B, 0.0))
+    work.append(("select", 1, N * 4 * 2 + R * 3 * 4, 0.0))
     work.append(("row_norm", 1, R * D * (4 + 4 + e), 0.0))
     for kc in ("gemm_qkv", "attn_ragged", "gemm_o", "gemm_gateup", "gemm_down"):
         by, fl = algorithmic_work(kc, case, R, kept_per_req, plen)
@@ -466,6 +471,113 @@ def run_block_mode(args, case, dev, world, barrier):
     ctx.close()
 
 
+# ------------------------------------------------------------------ a trace through the scheduler
+class _DenseEngine:
+    """A plain block-diffusion engine for comparison: every step of every block keeps the whole block."""
+
+    def __init__(self, engine):
+        self.engine = engine
+
+    def capacity_check(self, slots, block):
+        self.engine.capacity_check(slots, block)
+
+    def step(self, view, dense):
+        self.engine.step(view, True)
+
+    def commit(self, view):
+        self.engine.commit(view)
+
+
+def run_schedule_mode(args, case, dev, world, barrier):
+    """Continuous batching of a request trace through the effective-batch scheduler (host loop around
+    focus_step / focus_commit_block): 2N requests of the workload's model and prefix distribution, one or two
+    blocks each, arriving a few per iteration, over N slots and the row budget of a dense engine on N
+    requests (N x B).  Run twice on this GPU: with focused steps (a focused request costs k_max rows, so more
+    requests share the budget) and with a dense engine (every step keeps the whole block, every request
+    costs B rows).  tokens/s = block positions decoded / device time of the whole trace (the scheduler reads
+    the mask state after every iteration, so host work is inside that time)."""
+    from decodability_aware_token_b200 import FocusContext, StepParams
+    from decodability_aware_token_b200.scheduler import EffectiveBatchScheduler, FocusEngine, Request
+    w, shp = case.work, case.shape
+    N, B = w.n_requests, w.block
+    pool0, table, plen = case.batch["kv_pool"], case.batch["page_table"].cpu(), case.batch["prefix_len"].cpu()
+    S = int(pool0.shape[4])
+    n_req = 2 * N
+    g = torch.Generator().manual_seed(7)
+    src = torch.randint(0, N, (n_req,), generator=g).tolist()            # prompt of request r: that of src[r]
+    nblk = (1 + torch.randint(0, 2, (n_req,), generator=g)).tolist()
+    arrive = [r // max(1, N // 4) for r in range(n_req)]
+    max_pages = max(-(-(int(plen[b]) + 2 * B) // S) for b in range(N)) + 1
+    # requests share their source's full prompt pages (read only); a partly filled last page receives the
+    # first committed positions, so every request gets its own copy of it
+    n0 = int(pool0.shape[0])
+    prompt_pages, copies = [], []
+    for r in range(n_req):
+        b = src[r]
+        n_pg = -(-int(plen[b]) // S)
+        pg = table[b, :n_pg].tolist()
+        if int(plen[b]) % S:
+            copies.append(pg[-1])
+            pg[-1] = n0 + len(copies) - 1
+        prompt_pages.append(pg)
+    spare = n_req * (-(-2 * B // S) + 1)
+    extra = torch.zeros((len(copies) + spare,) + tuple(pool0.shape[1:]), dtype=pool0.dtype, device=pool0.device)
+    if copies:
+        extra[: len(copies)] = pool0[torch.tensor(copies, device=pool0.device)]
+    pool_init = torch.cat([pool0, extra], 0)
+    free0 = list(range(n0 + len(copies), int(pool_init.shape[0])))
+    params = StepParams(w.tau, w.k_min, w.k_max, w.conf_threshold, w.alpha)
+
+    def trace(dense: bool):
+        pool = pool_init.clone()
+        reqs = [Request(r, arrive[r], int(plen[src[r]]), prompt_pages[r], nblk[r]) for r in range(n_req)]
+        with FocusContext(shp, case.model, max_requests=N, max_block=B, max_keep=B,
+                          max_pages_per_req=max_pages) as ctx:
+            eng = FocusEngine(ctx, params)
+            sch = EffectiveBatchScheduler(_DenseEngine(eng) if dense else eng, slots=N, block=B,
+                                          n_layers=shp.n_layers, n_kv_heads=shp.n_kv_heads, head_dim=shp.head_dim,
+                                          max_pages_per_req=max_pages, kv_pool=pool, free_pages=free0,
+                                          mask_token=shp.vocab - 1, k_max=B if dense else w.k_max,
+                                          row_budget=N * B, keep_pages=True)
+            for rq in reqs:
+                sch.submit(rq)
+            torch.cuda.synchronize(dev)
+            barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            sch.run(max_iterations=100_000)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1)
+        decoded = sum(nblk) * B
+        return ms, decoded, sch.iteration, max(st.active for st in sch.stats)
+
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    time.sleep(0.3)
+    tw0 = time.time()
+    f_ms, f_tok, f_it, f_peak = trace(False)
+    d_ms, d_tok, d_it, d_peak = trace(True)
+    tw1 = time.time()
+    sampler.stop()
+    f_max, f_total = reduce_over_ranks(f_ms, f_tok, world, dev)
+    d_max, d_total = reduce_over_ranks(d_ms, d_tok, world, dev)
+    if int(os.environ.get("RANK", "0")) == 0:
+        line = {
+            "metric": "decoded tokens/s over a request trace (effective-batch scheduler, focused vs dense steps)",
+            "value": whole_job_rate(f_total, f_max), "unit": UNIT, "n_gpus": world, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": shp.dtype, "data": "synthetic",
+            "dense_engine": {"value": whole_job_rate(d_total, d_max), "ms": d_max, "iterations": d_it,
+                             "max_active": d_peak},
+            "focused": {"ms": f_max, "iterations": f_it, "max_active": f_peak},
+            "speedup_vs_dense": (d_max / f_max) if f_max > 0 else None,
+            "clocks": sampler.summary(tw0, tw1),
+            "config": {"workload": args.workload, "mode": "schedule", "desc": workload_desc(case),
+                       "requests": n_req, "slots": N, "row_budget": N * B, "blocks": sum(nblk),
+                       "launch": "eager calls; the scheduler reads the mask state after every iteration"},
+        }
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ the GPU arm
 def main():
     args = parse()
@@ -492,8 +604,8 @@ def main():
     case = make_workload(args, rank_seed(base, rank), dev)    # this rank's requests
     w, shp = case.work, case.shape
     N, B = w.n_requests, w.block
-    if args.mode == "block":
-        run_block_mode(args, case, dev, world, barrier)
+    if args.mode in ("block", "schedule"):
+        (run_block_mode if args.mode == "block" else run_schedule_mode)(args, case, dev, world, barrier)
         if world > 1:
             dist.destroy_process_group()
         return

@@ -10,9 +10,12 @@
 // written ascending.  Forced fraction f >= 0: k = min(B, ceil(f B)) over all positions under
 // (masked first, delta desc, j asc).
 //
-// One CTA: a warp per request (B <= 64: each lane owns positions lane and lane + 32), ballots for the
-// counts, an O(B) rank per position (B^2 <= 4096 compares per request), then a serial exclusive scan of
-// the kept counts and the row map.  The work is a few KB, so the kernel is latency-bound by design.
+// Two kernels.  select_kernel: a warp per request, eight requests per CTA (B <= 64: each lane owns positions
+// lane and lane + 32): the request's importance partials summed in group order, ballots for the counts, an
+// O(B) rank per position (B^2 <= 4096 compares per request), the kept positions written ascending.
+// rowmap_kernel: one CTA scans the kept counts (block-wide, in order of requests) into the row offsets and
+// writes the ragged row map.  Both are latency-bound; spreading the requests over CTAs keeps the read of
+// the importance partials (4 MB at 256 requests of block 64 with 32 groups) parallel.
 #include "launch.h"
 
 namespace focus {
@@ -25,17 +28,17 @@ __device__ __forceinline__ bool key_less(bool forced, bool ma, float da, int ja,
     return ja < jb;                     // lower position first
 }
 
-__global__ void __launch_bounds__(1024) select_kernel(SelectArgs a) {
+constexpr int kSelWarps = 8;  // requests per select CTA
+
+__global__ void __launch_bounds__(32 * kSelWarps) select_kernel(SelectArgs a) {
     pdl_entry();
-    extern __shared__ int32_t sh[];  // [N] kept counts, [N + 1] offsets
-    int32_t* kc_s = sh;
-    int32_t* off_s = sh + a.N;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int B = a.B;
     const bool forced = a.forced_frac >= 0.f;
     const size_t layer_stride = (size_t)a.N * a.groups * B;
 
-    for (int b = warp; b < a.N; b += nw) {
+    const int b = blockIdx.x * kSelWarps + warp;
+    if (b < a.N) {
         float dl[2];
         bool valid[2], msk[2], keep[2];
         for (int h = 0; h < 2; ++h) {
@@ -112,44 +115,73 @@ __global__ void __launch_bounds__(1024) select_kernel(SelectArgs a) {
         if (keep[0]) ret[__popc(lo & lt)] = lane;
         if (keep[1]) ret[__popc(lo) + __popc(hi & lt)] = lane + 32;
         for (int t = kept + lane; t < a.max_keep; t += 32) ret[t] = -1;
-        if (lane == 0) {
-            a.keep_count[b] = kept;
-            kc_s[b] = kept;
-        }
+        if (lane == 0) a.keep_count[b] = kept;
     }
+}
+
+// Exclusive scan of the kept counts (requests in order) into row_offsets and the live row count, then the
+// row map: compacted row row_offsets[b] + t is position retained_idx[b][t] of request b.
+__global__ void __launch_bounds__(1024) rowmap_kernel(SelectArgs a) {
+    pdl_entry();
+    __shared__ int32_t warp_sum[32];
+    __shared__ int32_t carry_s;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) carry_s = 0;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int off = 0;
-        for (int b = 0; b < a.N; ++b) {
-            off_s[b] = off;
-            a.row_offsets[b] = off;
-            off += kc_s[b];
+    for (int base = 0; base < a.N; base += 1024) {
+        const int b = base + tid;
+        const int v = b < a.N ? a.keep_count[b] : 0;
+        int inc = v;  // inclusive scan within the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
         }
-        off_s[a.N] = off;
-        a.row_offsets[a.N] = off;
-        *a.n_rows = off;
+        if (lane == 31) warp_sum[warp] = inc;
+        __syncthreads();
+        if (warp == 0) {
+            int w = warp_sum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_sum[lane] = w;  // inclusive over warps
+        }
+        __syncthreads();
+        const int carry = carry_s;
+        if (b < a.N) a.row_offsets[b] = carry + (warp > 0 ? warp_sum[warp - 1] : 0) + inc - v;
+        __syncthreads();
+        if (tid == 0) carry_s = carry + warp_sum[31];
+        __syncthreads();
     }
-    __syncthreads();
-    for (int b = warp; b < a.N; b += nw) {
-        const int base = off_s[b], k = kc_s[b];
+    if (tid == 0) {
+        a.row_offsets[a.N] = carry_s;
+        *a.n_rows = carry_s;
+    }
+    __syncthreads();  // the offsets this CTA wrote are visible to all of its threads
+    for (int b = warp; b < a.N; b += 32) {
+        const int off = a.row_offsets[b], k = a.keep_count[b];
         for (int t = lane; t < k; t += 32) {
             const int j = a.retained_idx[(size_t)b * a.max_keep + t];
-            a.row_req[base + t] = b;
-            a.row_pos[base + t] = j;
-            a.row_src[base + t] = b * B + j;
+            a.row_req[off + t] = b;
+            a.row_pos[off + t] = j;
+            a.row_src[off + t] = b * a.B + j;
         }
     }
 }
 
 }  // namespace
 
-bool configure_select_kernel() { return max_shared_carveout((const void*)select_kernel); }
+bool configure_select_kernel() {
+    return max_shared_carveout((const void*)select_kernel) && max_shared_carveout((const void*)rowmap_kernel);
+}
 
 int launch_select(const SelectArgs& a, cudaStream_t s) {
     if (a.N <= 0) return 0;
-    const size_t smem = sizeof(int32_t) * (2 * (size_t)a.N + 1);
-    if (smem > 48 * 1024) cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    return launched(launch_pdl(select_kernel, dim3(1), dim3(1024), smem, s, 0, a));
+    const dim3 grid((a.N + kSelWarps - 1) / kSelWarps);
+    if (launch_pdl(select_kernel, grid, dim3(32 * kSelWarps), 0, s, 0, a) != cudaSuccess) return -1;
+    return launch_pdl(rowmap_kernel, dim3(1), dim3(1024), 0, s, 0, a) == cudaSuccess ? 2 : -1;
 }
 
 }  // namespace focus
