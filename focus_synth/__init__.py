@@ -14,7 +14,8 @@ Overview -- Motivation and Runtime Action: a block of B tokens is denoised at
 each step on top of an exactly cached prefix.
 
 Recipe (all seeded; every tensor gets its own generator seeded from
-(base seed, tensor name, layer), so generation order does not matter):
+(base seed, tensor name, layer), so generation order does not matter; tensors of more than 2^30
+elements are drawn in 2^28-element slices with one generator per slice):
   * weights  ~ N(0, 0.02), norms gamma ~ 1 + N(0, 0.1), embeddings ~ N(0, 1),
     rounded to the model dtype (bf16, or fp32 for the tiny model);
   * prefix KV pages and the intra-block KV cache ~ N(0, 1), model dtype;
@@ -90,6 +91,9 @@ MODEL_SHAPES = {
     "small_bf16": ModelShape(4, 512, 8, 4, 128, 1536, 4000, "bf16"),
     "small_bf16_g4": ModelShape(3, 512, 8, 2, 128, 1024, 2100, "bf16"),
     "small_f32": ModelShape(3, 256, 4, 2, 64, 768, 700, "f32"),
+    # hidden 2048 with enough block rows that the many-row GEMMs run on the persistent kernel, still
+    # small enough (3 layers, vocabulary 4096) for the oracle
+    "wide_bf16": ModelShape(3, 2048, 16, 8, 128, 3072, 4096, "bf16"),
 }
 
 WORKLOADS = {
@@ -100,13 +104,14 @@ WORKLOADS = {
     # reduced workloads for parity at oracle-friendly sizes
     "small": Workload(5, 32, 64, ("uniform", 0, 300), ("frac", 0.3, 1.0), k_min=1, k_max=8),
     "small_b16": Workload(6, 16, 16, ("uniform", 0, 90), ("frac", 0.0, 1.0), k_min=2, k_max=6),
+    "wide": Workload(41, 64, 64, ("uniform", 0, 600), ("frac", 0.3, 1.0), k_min=1, k_max=16),
 }
 
 # seed of each named case: 1234 + the workload's index among the five
 # workloads (tiny, 1.7B N32, 1.7B N128, 8B N256, 1.7B sweep); reduced cases from 2001
 SEEDS = {
     "tiny": 1235, "sdar1.7b_n32_b32": 1236, "sdar1.7b_n128_b32": 1237, "sdar8b_n256_b64": 1238,
-    "sweep": 1239, "small_bf16": 2001, "small_bf16_g4": 2002, "small_f32": 2003,
+    "sweep": 1239, "small_bf16": 2001, "small_bf16_g4": 2002, "small_f32": 2003, "wide_bf16": 2004,
 }
 
 # named cases: (model shape, workload)
@@ -118,6 +123,7 @@ CASES = {
     "small_bf16": ("small_bf16", "small"),
     "small_bf16_g4": ("small_bf16_g4", "small_b16"),
     "small_f32": ("small_f32", "small_b16"),
+    "wide_bf16": ("wide_bf16", "wide"),
 }
 
 
@@ -151,14 +157,35 @@ def _gen(device, seed):
     return g
 
 
+_SLICE = 1 << 28  # elements drawn per generator for very large tensors
+
+
 def _normal(shape, std, mean, seed, device, dtype):
-    g = _gen(device, seed)
-    t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
-    if std != 1.0:
-        t.mul_(std)
-    if mean != 0.0:
-        t.add_(mean)
-    return t.to(dtype)
+    """N(mean, std^2) in float32, rounded to `dtype`.  Tensors of more than 2^30 elements (the page pools of
+    the full-size workloads) are drawn in slices of 2^28 elements, each from its own generator seeded from
+    (seed, slice index), straight into the result: the float32 draw of a whole 60 GB page pool would not fit
+    on the device next to it."""
+    n = math.prod(shape)
+    if n <= (1 << 30):
+        g = _gen(device, seed)
+        t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+        if std != 1.0:
+            t.mul_(std)
+        if mean != 0.0:
+            t.add_(mean)
+        return t.to(dtype)
+    out = torch.empty(shape, dtype=dtype, device=device)
+    flat = out.view(-1)
+    for i, lo in enumerate(range(0, n, _SLICE)):
+        hi = min(n, lo + _SLICE)
+        g = _gen(device, _seed_of(seed, "slice", i))
+        t = torch.randn(hi - lo, generator=g, device=device, dtype=torch.float32)
+        if std != 1.0:
+            t.mul_(std)
+        if mean != 0.0:
+            t.add_(mean)
+        flat[lo:hi].copy_(t)
+    return out
 
 
 def make_model(shape: ModelShape, seed: int, device="cpu", lm_boost_rows: Optional[torch.Tensor] = None,

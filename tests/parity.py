@@ -1,9 +1,10 @@
 """Tie-aware comparison of a GPU focused step against the CPU oracle.
 
 Which oracle a case is compared with:
-  * the float32 path, and the bf16 path on shallow models (at most 4 layers): the plain float64 oracle,
-    for values and decisions alike, with no allowance;
-  * the bf16 path on deep models (the 28- and 36-layer shapes): values against the float64 oracle with
+  * the float32 path, and the bf16 path on shallow, narrow models (at most 4 layers, hidden at most 1024):
+    the plain float64 oracle, for values and decisions alike, with no allowance;
+  * the bf16 path on deep or wide models (the 28- and 36-layer shapes; hidden 2048, where a bf16 evaluation
+    already drifts 1.5 % of RMS at 4 layers): values against the float64 oracle with
     an allowance of twice the drift that bf16 storage alone causes (see below), decisions against the
     oracle run with bf16 storage at the kernel's storage points ("decision oracle"); agreement of the
     decisions with the float64 oracle at 1e-3 gates is counted and reported (decision_report).
@@ -22,9 +23,12 @@ Rules (what is unique is compared exactly, what is not is checked for validity):
     drift of bf16 storage (bf16-storage oracle minus float64 oracle, per quantity); the RMS of the error
     <= frac x RMS plus, for deep bf16 cases, twice the RMS of that drift;
   * kept set per request: identical wherever the oracle's delta gap at the top-k cut and its
-    |delta - tau| both exceed the selection gate (1e-3); otherwise the GPU set must still be a valid
-    top-k of the oracle's deltas within that gate (and the test then re-runs the GPU with the oracle's
-    set forced to compare everything downstream);
+    |delta - tau| both exceed the selection gate; otherwise the GPU set must still be a valid top-k of
+    the oracle's deltas within that gate (and the test then re-runs the GPU with the oracle's set forced
+    to compare everything downstream).  The gate is 1e-3 for the float32 path; on the bf16 path it is,
+    per request, the larger of 1e-3 and twice the largest |delta| change that bf16 storage alone makes to
+    that request (the argument of the value allowance: two valid bf16 evaluations of layers 0-1 differ by
+    about that much; at hidden 4096, or with large importance values, it exceeds 1e-3);
   * top id per kept row: identical where the oracle's top-1 logit margin exceeds the logit gate;
     otherwise the GPU's id must be within the gate of the oracle's best logit.  For bf16 the gate is the
     logit error that the hidden-state tolerance allows (frac x sqrt(D) x RMS of the LM-head weights,
@@ -147,12 +151,20 @@ def drift_allowance(ora: fo.OracleResult, ora_exact: fo.OracleResult) -> dict:
     return out
 
 
+def selection_gates(ora: fo.OracleResult, ora_exact: fo.OracleResult, gate: float) -> np.ndarray:
+    """Per request: max(gate, twice the largest |delta| change that bf16 storage alone makes)."""
+    drift = np.abs(ora.delta - ora_exact.delta).max(axis=1) if ora.delta.size else np.zeros(0)
+    return np.maximum(gate, 2.0 * drift)
+
+
 def compare(case, params: dict, ora: fo.OracleResult, gpu: dict, tol: Tol, ibc_in, check_selection=True,
-            allow=None):
+            allow=None, sel_gates=None):
     """Assert parity; returns (report dict, list of requests whose kept set differs within the gate)."""
     report = {}
     allow = allow or {}
     N, B = ora.decoded_ids.shape
+    gates = np.full(N, tol.sel) if sel_gates is None else np.asarray(sel_gates, dtype=np.float64)
+    report["sel_gate_max"] = float(gates.max()) if N else tol.sel
     logit_gate = tol.logit if tol.logit is not None else \
         derived_logit_gate(case, tol.frac + allow.get("hidden_rel", 0.0))
     lc_gate = tol.log_conf if tol.log_conf is not None else 2 * logit_gate
@@ -170,10 +182,10 @@ def compare(case, params: dict, ora: fo.OracleResult, gpu: dict, tol: Tol, ibc_i
         assert kg == sorted(kg), f"request {b}: kept positions not ascending"
         if kg == ko:
             continue
-        exact = ora.cut_gap[b] > tol.sel and ora.tau_gap[b] > tol.sel
-        assert check_selection and not exact, (f"request {b}: kept {kg} vs oracle {ko} "
-                                               f"(cut gap {ora.cut_gap[b]:.2e}, tau gap {ora.tau_gap[b]:.2e})")
-        assert valid_selection(kg, ora.delta[b], masked0[b], params, tol.sel, B), \
+        exact = ora.cut_gap[b] > gates[b] and ora.tau_gap[b] > gates[b]
+        assert check_selection and not exact, (f"request {b}: kept {kg} vs oracle {ko} (cut gap "
+                                               f"{ora.cut_gap[b]:.2e}, tau gap {ora.tau_gap[b]:.2e}, gate {gates[b]:.2e})")
+        assert valid_selection(kg, ora.delta[b], masked0[b], params, gates[b], B), \
             f"request {b}: kept {kg} is not a valid top-k within the gate (oracle {ko})"
         flipped.append(b)
     off = _np(gpu["row_offsets"])

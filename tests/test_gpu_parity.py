@@ -65,6 +65,16 @@ def test_alpha_tau_kmin_variants(name):
     check(case, step_params(case.work, alpha=0.5, tau=-0.01, k_min=0, k_max=case.work.k_max), m)
 
 
+@pytest.mark.parametrize("frac", [-1.0, 1.0])
+def test_many_row_gemms_match_oracle(frac):
+    """Hidden 2048, 41 requests of block 64: the 2624 block rows (a ragged last 128-row tile) give the
+    layers-0-1 GEMMs enough tiles for the persistent kernel, with 256-wide tiles for some GEMMs and 128-wide
+    for others.  Adaptive: the kept rows (up to 656) run on the one-tile-per-CTA kernel; keep fraction 1:
+    the last layer's 2624 kept rows run on the persistent kernel too."""
+    case = _case("wide_bf16")
+    check(case, step_params(case.work, forced_keep_frac=frac), _model("wide_bf16", case))
+
+
 def _with_batch(case, **fields):
     b = dict(case.batch)
     b.update(fields)
@@ -262,16 +272,22 @@ def pick_requests(case, gpu, params, n):
 
 def _sampled_check(case, n_requests=8, params=None):
     """Full-size case on the GPU (model, pages and cache stay on the device); the oracle runs only the
-    chosen requests (requests are independent) and reads their pages from the device."""
+    chosen requests (requests are independent) and reads their pages from the device.  The case's device
+    tensors are released on the way out, pass or fail (a failure's traceback would keep them alive)."""
     p = params or step_params(case.work)
-    gpu = run_gpu(case, p, case.model)
-    host = fs.Case(case.shape, case.work, case.model, {k: (v if k == "kv_pool" else v.cpu()) for k, v in case.batch.items()},
-                   case.seed)
-    reqs = pick_requests(host, gpu, p, n_requests)
-    rep = check(host, p, requests=reqs, gpu=gpu)
-    rep["checked"] = reqs
-    del gpu, host
-    return rep
+    host_batch = {}
+    try:
+        gpu = run_gpu(case, p, case.model)
+        host_batch.update({k: (v if k == "kv_pool" else v.cpu()) for k, v in case.batch.items()})
+        host = fs.Case(case.shape, case.work, case.model, host_batch, case.seed)
+        reqs = pick_requests(host, gpu, p, n_requests)
+        rep = check(host, p, requests=reqs, gpu=gpu)
+        rep["checked"] = reqs
+        return rep
+    finally:
+        host_batch.clear()
+        case.batch.clear()
+        case.model.clear()
 
 
 @pytest.mark.slow
