@@ -1,0 +1,452 @@
+// bf16 attention of block queries over paged prefix KV plus the intra-block KV cache on the 5th-generation
+// tensor cores (tcgen05.mma with S and O accumulators in TMEM), with the importance column sums fused in
+// for layers 0 and 1.  Used for launches whose (request, KV head) units hold more than 32 query vectors --
+// many kept rows, or four query heads per KV head -- where the legacy mma.sync kernel (attention_tc.cu)
+// runs out of tensor throughput before it runs out of memory bandwidth.
+//
+// "FOCUS: DLLMs Know How to Tame Their Compute Bound", project page, Overview -- Design / Decodability
+// Signal (importance from the early layers' Q/K attention) and Runtime Action (ragged execution and the
+// intra-block KV cache); news article on the same paper, "Arquitetura do FOCUS" (ragged paged attention).
+//
+// Work unit (one CTA): request b, KV head g and a tile of up to 128 query vectors of that group (query
+// vector qi = row * G + head-in-group; the tile is the MMA's M = 128).  Keys are walked in 64-key chunks:
+// the prefix pages in order, then the B block keys from the intra-block cache as the last chunk (the same
+// TMA chunk loads as the mma.sync kernel).  Per chunk i:
+//   S_i = Q K_i^T         tcgen05.mma M = 128, N = 64, K = 128 (both operands K-major), into one of two
+//                         64-column TMEM buffers, issued before the softmax of chunk i - 1 has finished;
+//   softmax (4 warps, one query vector per thread): S_i from TMEM, masked and scaled to base 2, online
+//                         max / denominator; P_i = 2^(s - m) rounded to bf16 into one of two shared buffers;
+//   O += P_i V_i          tcgen05.mma M = 128, N = 128, K = 64, V taken MN-major straight from the page
+//                         tile, into a 128-column TMEM accumulator.
+// The running max m is raised only when a chunk exceeds it by more than 8 (a factor of 256 in the
+// weights); O and the denominator are then rescaled in TMEM.  Between raises, weights up to 2^8 are
+// summed exactly as the plain online softmax would sum them after its rescale, so the result is the same
+// softmax.  Warp roles: warp 0 lane 0 issues the TMA copies, warp 1 owns TMEM and its lane 0 issues the
+// MMAs, warps 2..5 run the softmax and the output.
+//
+// Importance: the block chunk's scaled scores stay in registers until the final m and denominator are
+// known; the probabilities of the block keys are then summed over the tile's query vectors per key in
+// fixed order (through shared memory) into imp_part[b][g][tile][j]; the selection kernel adds those in order.
+//
+// Every mbarrier wait is bounded; on expiry the role flags FOCUS_DEVERR_TIMEOUT and stops, the producer
+// waits (bounded) for its own copies, the MMA thread for its own MMAs, and TMEM is released after both.
+#include <math_constants.h>
+
+#include "attention_pages.cuh"
+
+namespace focus {
+
+namespace {
+
+using tc::idesc_bf16;
+using tc::mbar_arrive;
+using tc::mma_bf16;
+using tc::mma_commit;
+using tc::smem_desc_sw128;
+using tc::smem_u32;
+using tc::tc_fence_after;
+using tc::tc_fence_before;
+using tc::tmem_ld32;
+
+constexpr int kT5Q = 128;                         // query vectors per CTA (MMA M)
+constexpr int kT5Stages = 3;                      // K/V chunks in the ring
+constexpr int kT5QHalf = kT5Q * 128;              // [128 q][64 d] bf16: 16 KB
+constexpr int kT5PBytes = kT5Q * 128;             // [128 q][64 keys] bf16: 16 KB
+constexpr int kT5Smem = 2 * kT5QHalf + kT5Stages * kStageBytes + 2 * kT5PBytes + 1024;  // 161 KB
+constexpr uint32_t kT5TmemCols = 256;             // S (two 64-column buffers) + O (128 columns)
+constexpr uint32_t kT5OCol = 128;                 // first TMEM column of O
+constexpr float kT5Raise = 8.f;                   // base-2 headroom before the running max is raised
+
+// 3-D TMA load (q rows: d, head, row).
+__device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* bar, void* dst, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes, written back.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    uint32_t r[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory descriptor of an MN-major operand written by TMA with the 128-byte swizzle: 64 elements of
+// the MN dimension per 128-byte row, consecutive K indices on consecutive rows; the next 64 MN elements
+// `lbo` bytes on, the next 8 K rows 1024 bytes on.
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t addr, uint32_t lbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFF);        // start address
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;   // leading byte offset: next 64 MN elements
+    d |= (uint64_t)(1024 >> 4) << 32;             // stride byte offset: next 8 K rows
+    d |= (uint64_t)1 << 46;                       // descriptor version for tcgen05
+    d |= (uint64_t)2 << 61;                       // 128-byte swizzle
+    return d;
+}
+
+template <bool FULL>
+__global__ void __launch_bounds__(192, 1) attention_t5_kernel(const __grid_constant__ CUtensorMap pool_map,
+                                                              const __grid_constant__ CUtensorMap ibc_map,
+                                                              const __grid_constant__ CUtensorMap q_map, AttnArgs a,
+                                                              int q_tiles) {
+    pdl_trigger();
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* q_s = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* kv_s = q_s + 2 * kT5QHalf;
+    uint8_t* p_s = kv_s + kT5Stages * kStageBytes;
+    __shared__ __align__(8) uint64_t q_full;
+    __shared__ __align__(8) uint64_t kv_full[kT5Stages];
+    __shared__ __align__(8) uint64_t kv_empty[kT5Stages];
+    __shared__ __align__(8) uint64_t s_full[2];
+    __shared__ __align__(8) uint64_t s_free[2];
+    __shared__ __align__(8) uint64_t p_full[2];
+    __shared__ __align__(8) uint64_t pv_bar;
+    __shared__ __align__(8) uint64_t done_bar;
+    __shared__ uint64_t valid_s[kT5Stages];
+    __shared__ int32_t pt_s[kPtCache];
+    __shared__ uint32_t tmem_slot;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = a.Hq / a.Hkv;
+    Unit u{};
+    u.b = blockIdx.x;
+    u.g = blockIdx.y;
+    u.qt = blockIdx.z;
+    u.P = checked_prefix(a.prefix_len, u.b, a.max_pages * a.page_size, a.err);
+    u.q0 = u.qt * kT5Q;
+    const int n_prefix_chunks = (u.P + kChunk - 1) / kChunk;
+    const int n_chunks = n_prefix_chunks + 1;
+    const int unit = (u.b * a.Hkv + u.g) * q_tiles + u.qt;
+
+    const bool pt_cached = a.max_pages <= kPtCache;
+    for (int i = threadIdx.x; pt_cached && i < a.max_pages; i += blockDim.x)
+        pt_s[i] = a.page_table[(size_t)u.b * a.max_pages + i];
+    const int32_t* pt = pt_cached ? pt_s : a.page_table + (size_t)u.b * a.max_pages;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&q_full, 1);
+        for (int s = 0; s < kT5Stages; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&s_free[b], 4);  // one arrival per softmax warp
+            mbar_init(&p_full[b], 4);
+        }
+        mbar_init(&pv_bar, 1);
+        mbar_init(&done_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                     "r"(kT5TmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    pdl_wait();
+
+    if (FULL) {
+        u.row_base = u.b * a.B;
+        u.n_rows = a.B;
+    } else {
+        u.row_base = a.row_offsets[u.b];
+        u.n_rows = a.row_offsets[u.b + 1] - u.row_base;
+    }
+    u.nq = min(kT5Q, u.n_rows * G - u.q0);
+    if (u.nq > 0) {
+        if (warp == 0) {
+            if (lane == 0) {
+                // ---- TMA producer: the query tile once, then the key / value chunks through the ring
+                asm volatile("prefetch.tensormap [%0];" ::"l"(&q_map) : "memory");
+                mbar_expect_tx(&q_full, 2u * kT5QHalf);
+                const int row0 = u.row_base + u.q0 / G;
+                tma_load_3d(&q_map, &q_full, q_s, 0, u.g * G, row0);
+                tma_load_3d(&q_map, &q_full, q_s + kT5QHalf, 64, u.g * G, row0);
+                int issued = 0;
+                for (int i = 0; i < n_chunks; ++i) {
+                    const int st = i % kT5Stages;
+                    if (!mbar_wait(&kv_empty[st], ((uint32_t)(i / kT5Stages) & 1u) ^ 1u, a.err)) break;
+                    valid_s[st] = issue_chunk(a, u, &pool_map, &ibc_map, kv_s + st * kStageBytes, &kv_full[st], i,
+                                              n_prefix_chunks, pt);
+                    ++issued;
+                }
+                // never leave with copies in flight
+                mbar_wait(&q_full, 0u, a.err);
+                for (int i = issued > kT5Stages ? issued - kT5Stages : 0; i < issued; ++i)
+                    mbar_wait(&kv_full[i % kT5Stages], (uint32_t)(i / kT5Stages) & 1u, a.err);
+            }
+            __syncwarp();
+        } else if (warp == 1) {
+            if (lane == 0) {
+                // ---- MMA issuer: S_i, then P_{i-1} V_{i-1}, so the S of the next chunk overlaps the softmax
+                constexpr uint32_t idesc_s = idesc_bf16(128, 64);
+                constexpr uint32_t idesc_o = idesc_bf16(128, 128) | (1u << 16);  // B (V) MN-major
+                const uint32_t q_addr = smem_u32(q_s);
+                bool ok = mbar_wait(&q_full, 0u, a.err);
+                auto pv = [&](int j) {
+                    const int pb = j & 1, st = j % kT5Stages;
+                    if (!mbar_wait(&p_full[pb], (uint32_t)(j >> 1) & 1u, a.err)) return false;
+                    tc_fence_after();
+                    const uint32_t p_addr = smem_u32(p_s + pb * kT5PBytes);
+                    const uint32_t v_addr = smem_u32(kv_s + st * kStageBytes + 2 * kHalf);
+#pragma unroll
+                    for (int kk = 0; kk < kChunk / 16; ++kk)
+                        mma_bf16(tmem + kT5OCol, smem_desc_sw128(p_addr + kk * 32),
+                                 smem_desc_sw128_mn(v_addr + kk * 2048, kHalf), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&pv_bar);
+                    mma_commit(&kv_empty[st]);  // K and V of chunk j have been read
+                    return true;
+                };
+                int i = 0;
+                for (; ok && i < n_chunks; ++i) {
+                    const int st = i % kT5Stages, sb = i & 1;
+                    if (!mbar_wait(&kv_full[st], (uint32_t)(i / kT5Stages) & 1u, a.err) ||
+                        !mbar_wait(&s_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(kv_s + st * kStageBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk) {
+                        const uint32_t off = (uint32_t)((kk >> 2) * kHalf + (kk & 3) * 32);
+                        mma_bf16(tmem + (uint32_t)(sb * 64), smem_desc_sw128(q_addr + (uint32_t)((kk >> 2) * kT5QHalf) +
+                                                                             (uint32_t)((kk & 3) * 32)),
+                                 smem_desc_sw128(k_addr + off), idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&s_full[sb]);
+                    if (i >= 1 && !pv(i - 1)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (ok) pv(n_chunks - 1);
+                mma_commit(&done_bar);
+                mbar_wait(&done_bar, 0u, a.err);
+            }
+            __syncwarp();
+        } else {
+            // ---- softmax and output: one query vector per thread
+            const int quarter = warp & 3;
+            const int t = quarter * 32 + lane;                   // query vector within the tile
+            const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+            const float sl2 = rsqrtf((float)kD) * 1.4426950408889634f;  // 1/sqrt(d) * log2(e)
+            float m_used = -CUDART_INF_F, l = 0.f;
+            float sb[kChunk];                                    // block chunk: scaled scores (importance)
+            bool alive = true;
+            for (int i = 0; i < n_chunks; ++i) {
+                const int st = i % kT5Stages, sbuf = i & 1;
+                bool ok = mbar_wait(&s_full[sbuf], (uint32_t)(i >> 1) & 1u, a.err) &&
+                          mbar_wait(&kv_full[st], (uint32_t)(i / kT5Stages) & 1u, a.err);  // valid_s is written
+                if (!__all_sync(0xffffffffu, ok)) {
+                    alive = false;
+                    break;
+                }
+                tc_fence_after();
+                float s[kChunk];
+                tmem_ld32(trow + (uint32_t)(sbuf * 64), *reinterpret_cast<float(*)[32]>(s));
+                tmem_ld32(trow + (uint32_t)(sbuf * 64 + 32), *reinterpret_cast<float(*)[32]>(s + 32));
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[sbuf]);
+                const uint64_t vmask = valid_s[st];
+                float cmax = -CUDART_INF_F;
+#pragma unroll
+                for (int c = 0; c < kChunk; ++c) {
+                    s[c] = ((vmask >> c) & 1ull) ? s[c] * sl2 : -CUDART_INF_F;
+                    cmax = fmaxf(cmax, s[c]);
+                }
+                // P V of the previous chunk has completed: O is stable and P buffer i % 2 is free
+                if (i >= 1) {
+                    ok = mbar_wait(&pv_bar, (uint32_t)(i - 1) & 1u, a.err);
+                    if (!__all_sync(0xffffffffu, ok)) {
+                        alive = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                // raise the running max only by more than kT5Raise; O and the denominator follow it
+                float f = 1.f;
+                if (m_used == -CUDART_INF_F) {
+                    m_used = cmax;  // no weight has been summed yet: O and l are zero
+                } else if (cmax > m_used + kT5Raise) {
+                    f = exp2f(m_used - cmax);
+                    l *= f;
+                    m_used = cmax;
+                }
+                if (__any_sync(0xffffffffu, f != 1.f)) {  // TMEM access is warp-collective: factor 1 elsewhere
+#pragma unroll 1
+                    for (int c0 = 0; c0 < kD; c0 += 32) {
+                        float v[32];
+                        tmem_ld32(trow + kT5OCol + (uint32_t)c0, v);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) v[c] *= f;
+                        tmem_st32(trow + kT5OCol + (uint32_t)c0, v);
+                    }
+                }
+                const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;
+                float rs = 0.f;
+                uint32_t pk[kChunk / 2];
+#pragma unroll
+                for (int c = 0; c < kChunk; c += 2) {
+                    const float p0 = exp2f(s[c] - mu), p1 = exp2f(s[c + 1] - mu);
+                    rs += p0 + p1;
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                    pk[c / 2] = *reinterpret_cast<uint32_t*>(&b2);
+                }
+                l += rs;
+                if (FULL && i == n_chunks - 1) {
+#pragma unroll
+                    for (int c = 0; c < kChunk; ++c) sb[c] = s[c];
+                }
+                // P row t of buffer i % 2: 128 bytes, 16-byte chunk c at (c ^ (t & 7)) (the 128-byte swizzle)
+                uint8_t* prow = p_s + sbuf * kT5PBytes + (t >> 3) * 1024 + (t & 7) * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4*>(prow + ((c ^ (t & 7)) << 4)) =
+                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                // V rows of keys the copies left unfilled may hold stale bits: P is 0 there, so make V 0 too
+                if (vmask != ~0ull) {
+                    const int r = t & 63, h = t >> 6;
+                    if (!((vmask >> r) & 1ull)) {
+                        uint4* vr = reinterpret_cast<uint4*>(kv_s + st * kStageBytes + 2 * kHalf + h * kHalf + r * 128);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) vr[c] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[sbuf]);
+            }
+            // the last P V has completed: normalise and write this thread's query vector
+            if (alive) alive = __all_sync(0xffffffffu, mbar_wait(&pv_bar, (uint32_t)(n_chunks - 1) & 1u, a.err));
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const bool live = t < u.nq;
+            if (alive) {
+                tc_fence_after();
+                const int qi = u.q0 + t;
+                const int row = qi / G, hh = u.g * G + (qi - row * G);
+                bf16* dst = reinterpret_cast<bf16*>(a.o) + ((size_t)(u.row_base + row) * a.Hq + hh) * kD;
+#pragma unroll 1
+                for (int c0 = 0; c0 < kD; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(trow + kT5OCol + (uint32_t)c0, v);
+                    if (live) {
+#pragma unroll
+                        for (int c = 0; c < 32; c += 8) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(v[c + 2 * e] * inv, v[c + 2 * e + 1] * inv);
+                                w[e] = *reinterpret_cast<uint32_t*>(&b2);
+                            }
+                            *reinterpret_cast<uint4*>(dst + c0 + c) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+            }
+            if constexpr (FULL) {
+                if (a.imp_part != nullptr) {
+                    // column sums of the block keys' final probabilities over the tile's query vectors, in fixed
+                    // order through shared memory (the K / V ring is idle once the last P V completed).  Every
+                    // softmax warp reaches the named barrier, whether or not its waits succeeded; a timeout
+                    // contributes zeros (and the error word says the outputs are not valid).
+                    float* colbuf = reinterpret_cast<float*>(kv_s);  // [128 query vectors][65]
+                    const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;
+#pragma unroll
+                    for (int c = 0; c < kChunk; ++c)
+                        colbuf[t * 65 + c] =
+                            (alive && live && sb[c] != -CUDART_INF_F && l > 0.f) ? exp2f(sb[c] - mu) * inv : 0.f;
+                    tc::named_sync_epilogue();
+                    if (t < a.B) {
+                        float col = 0.f;
+                        for (int r = 0; r < kT5Q; ++r) col += colbuf[r * 65 + t];
+                        a.imp_part[(size_t)unit * a.B + t] = col;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kT5TmemCols) : "memory");
+}
+
+}  // namespace
+
+}  // namespace focus
+
+namespace focus {
+
+namespace {
+
+// 3-D view of the query rows for TMA: (d, query head, row), box (64, G, 128 / G): one box is the d half of
+// a 128-vector query tile of one KV group, laid out as 128 rows of 128 bytes with the 128-byte swizzle.
+bool make_q_map(CUtensorMap* m, const void* q, int rows_cap, int Hq, int G) {
+    auto fn = tc::encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)Hq, (cuuint64_t)rows_cap};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)Hq * kD * 2};
+    const cuuint32_t box[3] = {64u, (cuuint32_t)G, (cuuint32_t)(kT5Q / G)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool attention_t5_used(int q_rows, int G) { return q_rows * G > 32 && G >= 1 && G <= 16 && (G & (G - 1)) == 0; }
+
+int attention_t5_q_tiles(int q_rows, int G) { return (q_rows * G + kT5Q - 1) / kT5Q; }
+
+bool configure_attention_t5_kernels() {
+    return cudaFuncSetAttribute(attention_t5_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kT5Smem) ==
+               cudaSuccess &&
+           cudaFuncSetAttribute(attention_t5_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kT5Smem) ==
+               cudaSuccess &&
+           max_shared_carveout((const void*)attention_t5_kernel<true>) &&
+           max_shared_carveout((const void*)attention_t5_kernel<false>);
+}
+
+int launch_attention_t5(const AttnArgs& a, int q_tiles, cudaStream_t s) {
+    if (a.N <= 0 || q_tiles <= 0) return 0;
+    const int G = a.Hq / a.Hkv;
+    CUtensorMap pool_map, ibc_map, q_map;
+    const uint64_t ibc_rows = (uint64_t)a.N * a.L * 2 * a.Hkv * a.B;
+    if (!tc::make_map(&ibc_map, a.ibc, ibc_rows, kD, (uint32_t)a.B, false)) return -1;
+    if (a.n_pages > 0) {
+        const uint64_t pool_rows = (uint64_t)a.n_pages * a.L * 2 * a.Hkv * a.page_size;
+        if (!tc::make_map(&pool_map, a.kv_pool, pool_rows, kD, (uint32_t)a.page_size, false)) return -1;
+    } else {
+        pool_map = ibc_map;  // never used: with no pages every prefix key is invalid
+    }
+    if (!make_q_map(&q_map, a.q, a.q_rows_cap, a.Hq, G)) return -1;
+    const dim3 grid(a.N, a.Hkv, q_tiles);
+    if (a.row_offsets == nullptr)
+        return launched(launch_pdl(attention_t5_kernel<true>, grid, dim3(192), kT5Smem, s, 0, pool_map, ibc_map, q_map, a,
+                                   q_tiles));
+    return launched(launch_pdl(attention_t5_kernel<false>, grid, dim3(192), kT5Smem, s, 0, pool_map, ibc_map, q_map, a,
+                               q_tiles));
+}
+
+}  // namespace focus

@@ -24,7 +24,7 @@
 #include <math_constants.h>
 
 #include "launch.h"
-#include "tc_gemm_kernel.cuh"
+#include "attention_pages.cuh"
 
 namespace focus {
 
@@ -35,13 +35,8 @@ using tc::mbar_init;
 using tc::mbar_wait;
 using tc::tma_load_2d;
 
-constexpr int kChunk = 64;      // keys per chunk
-constexpr int kD = 128;         // head dim (bf16 path)
 constexpr int kQTile = 64;      // query vectors per CTA
 constexpr int kStages = 3;      // chunks in the ring (2 in flight while one is consumed)
-constexpr int kHalf = kChunk * 128;         // one [64 keys][64 d] bf16 half-tile: 8 KB
-constexpr int kStageBytes = 4 * kHalf;      // K lo, K hi, V lo, V hi: 32 KB
-constexpr int kPtCache = 512;               // page-table entries cached in shared memory
 constexpr int kAttnSmem = kStages * kStageBytes + 1024;  // dynamic shared memory: 97 KB, two CTAs per SM
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -75,60 +70,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&p);
-}
-
-struct Unit {
-    int b, g, qt, P, row_base, n_rows, nq, q0;
-};
-
-// Issue the TMA copies of chunk `ci` into stage `st` (one thread).  Prefix chunks copy whole pages
-// (64 / S pages, each as K and V halves); the last chunk copies the block's B cache rows.  Pages past
-// the prefix or with an out-of-range id are skipped (their keys stay masked).  Returns the valid-key
-// mask of the chunk.
-__device__ __forceinline__ uint64_t issue_chunk(const AttnArgs& a, const Unit& u, const CUtensorMap* pool_map,
-                                                const CUtensorMap* ibc_map, uint8_t* stage, uint64_t* bar, int ci,
-                                                int n_prefix_chunks, const int32_t* pt) {
-    const int S = a.page_size;
-    uint64_t mask = 0;
-    if (ci < n_prefix_chunks) {
-        uint32_t bytes = 0;
-        for (int p = 0; p < kChunk / S; ++p) {
-            const int t0 = ci * kChunk + p * S;
-            if (t0 >= u.P) break;
-            const int page = pt[t0 / S];
-            if (page < 0 || page >= a.n_pages) {
-                raise_err(a.err, FOCUS_DEVERR_PAGE_ID);
-                continue;
-            }
-            bytes += 4u * S * 128u;
-            const int n = min(S, u.P - t0);
-            mask |= (n == 64 ? ~0ull : ((1ull << n) - 1ull)) << (p * S);
-        }
-        mbar_expect_tx(bar, bytes);
-        for (int p = 0; p < kChunk / S; ++p) {
-            const int t0 = ci * kChunk + p * S;
-            if (t0 >= u.P) break;
-            const int page = pt[t0 / S];
-            if (page < 0 || page >= a.n_pages) continue;
-            const int krow = (int)(((((size_t)page * a.L + a.layer) * 2 + 0) * a.Hkv + u.g) * S);
-            const int vrow = krow + a.Hkv * S;
-            uint8_t* dst = stage + p * S * 128;
-            tma_load_2d(pool_map, bar, dst, 0, krow);
-            tma_load_2d(pool_map, bar, dst + kHalf, 64, krow);
-            tma_load_2d(pool_map, bar, dst + 2 * kHalf, 0, vrow);
-            tma_load_2d(pool_map, bar, dst + 3 * kHalf, 64, vrow);
-        }
-    } else {
-        const int krow = (int)(((((size_t)u.b * a.L + a.layer) * 2 + 0) * a.Hkv + u.g) * a.B);
-        const int vrow = krow + a.Hkv * a.B;
-        mbar_expect_tx(bar, 4u * a.B * 128u);
-        tma_load_2d(ibc_map, bar, stage, 0, krow);
-        tma_load_2d(ibc_map, bar, stage + kHalf, 64, krow);
-        tma_load_2d(ibc_map, bar, stage + 2 * kHalf, 0, vrow);
-        tma_load_2d(ibc_map, bar, stage + 3 * kHalf, 64, vrow);
-        mask = a.B == 64 ? ~0ull : ((1ull << a.B) - 1ull);
-    }
-    return mask;
 }
 
 template <bool FULL>
@@ -554,7 +495,7 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_const
 bool configure_attention_tc_kernels() {
     // once per context (device current): the shared-memory opt-in is not a stream operation, so it is
     // never made at launch time, where it would break stream capture
-    return cudaFuncSetAttribute(attention_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) ==
+    return configure_attention_t5_kernels() && cudaFuncSetAttribute(attention_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) ==
                cudaSuccess &&
            cudaFuncSetAttribute(attention_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) ==
                cudaSuccess &&
@@ -562,7 +503,9 @@ bool configure_attention_tc_kernels() {
            max_shared_carveout((const void*)attention_tc_kernel<false>);
 }
 
-int attention_q_tiles(int B, int G) { return (B * G + kQTile - 1) / kQTile; }
+int attention_q_tiles(int B, int G) {
+    return attention_t5_used(B, G) ? attention_t5_q_tiles(B, G) : (B * G + kQTile - 1) / kQTile;
+}
 
 bool attention_tc_page_size_ok(int S) { return S == 16 || S == 32 || S == 64; }
 
@@ -582,6 +525,7 @@ int attention_pieces(int units, int max_chunks) {
 
 int launch_attention_tc(const AttnArgs& a, int q_tiles, cudaStream_t s) {
     if (a.N <= 0 || q_tiles <= 0) return 0;
+    if (attention_t5_used(a.q_rows, a.Hq / a.Hkv)) return launch_attention_t5(a, q_tiles, s);
     // 2-D views for TMA: every (page, layer, K|V, head) block of S rows and every (request, layer,
     // K|V, head) cache block of B rows is a run of consecutive 256-byte rows
     CUtensorMap pool_map, ibc_map;

@@ -234,6 +234,7 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
     at.page_table = in->page_table; at.N = N; at.B = B; at.L = dm.L; at.Hq = dm.Hq; at.Hkv = dm.Hkv; at.d = dm.d;
     at.max_pages = c->lim.max_pages_per_req; at.page_size = in->page_size; at.n_pages = in->n_pages; at.err = c->err;
     at.part_o = c->att_part_o; at.part_ml = c->att_part_ml; at.sb_buf = c->att_sb; at.counters = c->att_counters;
+    at.q_rows_cap = c->lim.max_requests * c->lim.max_block;
     const int max_chunks = (c->lim.max_pages_per_req * in->page_size + 63) / 64 + 1;
     const int pieces_full = bf ? attention_pieces(N * dm.Hkv * qt_full, max_chunks) : 1;
     const int pieces_kept = bf ? attention_pieces(N * dm.Hkv * qt_kept, max_chunks) : 1;
@@ -260,6 +261,7 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
             });
         }
         at.layer = l;
+        at.q_rows = B;
         at.row_offsets = nullptr;
         at.imp_part = c->imp_part + (size_t)l * N * dm.Hkv * qt_full * B;
         at.pieces = pieces_full;
@@ -311,6 +313,7 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
             });
         }
         at.layer = l;
+        at.q_rows = k_cap;
         at.row_offsets = out->row_offsets;
         at.imp_part = nullptr;
         at.pieces = pieces_kept;

@@ -94,6 +94,8 @@ struct AttnArgs {
     float* part_ml;             // [unit * pieces + piece][64][2] partial row max / denominator (log2 domain)
     float* sb_buf;              // [unit][64][64] raw block-key scores (layers 0-1)
     int* counters;              // [unit] arrival counters, zero between launches
+    int q_rows;                 // bound on query rows per request in this launch (B, or the kept-row cap)
+    int q_rows_cap;             // rows the query buffer holds
 };
 
 constexpr int kAttnSplitCap = 1280;  // unit-pieces the split-KV scratch holds
@@ -105,6 +107,11 @@ template <typename T> int launch_attention(const AttnArgs& a, cudaStream_t s);
 // Returns the number of launches, or -1 if a tensor map could not be built.
 int launch_attention_tc(const AttnArgs& a, int q_tiles, cudaStream_t s);
 int attention_q_tiles(int B, int G);
+// tcgen05 kernel (attention_t5.cu) for units of more than 32 query vectors: 128-vector query tiles
+bool attention_t5_used(int q_rows, int G);
+int attention_t5_q_tiles(int q_rows, int G);
+int launch_attention_t5(const AttnArgs& a, int q_tiles, cudaStream_t s);
+bool configure_attention_t5_kernels();
 bool attention_tc_page_size_ok(int page_size);  // KV page sizes the TMA page loader handles: 16, 32, 64
 
 // ---- selection + compaction metadata (select.cu) ------------------------------
