@@ -15,7 +15,8 @@
 //   S_i = Q K_i^T         tcgen05.mma M = 128, N = 64, K = 128 (both operands K-major), into one of two
 //                         64-column TMEM buffers, issued before the softmax of chunk i - 1 has finished;
 //   softmax (4 warps, one query vector per thread): S_i from TMEM, masked and scaled to base 2, online
-//                         max / denominator; P_i = 2^(s - m) rounded to bf16 into one of two shared buffers;
+//                         max / denominator; P_i = 2^(s - m) rounded to bf16 into shared memory (one
+//                         buffer: the softmax of chunk i writes it only after P_{i-1} V_{i-1} completed);
 //   O += P_i V_i          tcgen05.mma M = 128, N = 128, K = 64, V taken MN-major straight from the page
 //                         tile, into a 128-column TMEM accumulator.
 // The running max m is raised only when a chunk exceeds it by more than 8 (a factor of 256 in the
@@ -49,10 +50,10 @@ using tc::tc_fence_before;
 using tc::tmem_ld32;
 
 constexpr int kT5Q = 128;                         // query vectors per CTA (MMA M)
-constexpr int kT5Stages = 3;                      // K/V chunks in the ring
+constexpr int kT5Stages = 4;                      // K/V chunks in the ring (three in flight while one is used)
 constexpr int kT5QHalf = kT5Q * 128;              // [128 q][64 d] bf16: 16 KB
 constexpr int kT5PBytes = kT5Q * 128;             // [128 q][64 keys] bf16: 16 KB
-constexpr int kT5Smem = 2 * kT5QHalf + kT5Stages * kStageBytes + 2 * kT5PBytes + 1024;  // 161 KB
+constexpr int kT5Smem = 2 * kT5QHalf + kT5Stages * kStageBytes + kT5PBytes + 1024;  // 177 KB
 constexpr uint32_t kT5TmemCols = 256;             // S (two 64-column buffers) + O (128 columns)
 constexpr uint32_t kT5OCol = 128;                 // first TMEM column of O
 constexpr float kT5Raise = 8.f;                   // base-2 headroom before the running max is raised
@@ -203,7 +204,7 @@ __global__ void __launch_bounds__(192, 1) attention_t5_kernel(const __grid_const
                     const int pb = j & 1, st = j % kT5Stages;
                     if (!mbar_wait(&p_full[pb], (uint32_t)(j >> 1) & 1u, a.err)) return false;
                     tc_fence_after();
-                    const uint32_t p_addr = smem_u32(p_s + pb * kT5PBytes);
+                    const uint32_t p_addr = smem_u32(p_s);
                     const uint32_t v_addr = smem_u32(kv_s + st * kStageBytes + 2 * kHalf);
 #pragma unroll
                     for (int kk = 0; kk < kChunk / 16; ++kk)
@@ -315,8 +316,8 @@ __global__ void __launch_bounds__(192, 1) attention_t5_kernel(const __grid_const
 #pragma unroll
                     for (int c = 0; c < kChunk; ++c) sb[c] = s[c];
                 }
-                // P row t of buffer i % 2: 128 bytes, 16-byte chunk c at (c ^ (t & 7)) (the 128-byte swizzle)
-                uint8_t* prow = p_s + sbuf * kT5PBytes + (t >> 3) * 1024 + (t & 7) * 128;
+                // P row t: 128 bytes, 16-byte chunk c at (c ^ (t & 7)) (the 128-byte swizzle)
+                uint8_t* prow = p_s + (t >> 3) * 1024 + (t & 7) * 128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
                     *reinterpret_cast<uint4*>(prow + ((c ^ (t & 7)) << 4)) =

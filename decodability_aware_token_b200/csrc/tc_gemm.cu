@@ -40,7 +40,7 @@ using namespace tc;
 // all rows beyond the live row count exit after the wait.
 constexpr int kBN = 128, kStages = 4;
 constexpr int kSmallRows = 256;  // GEMMs with at most this many rows run on the swapped kernel
-constexpr bool kUsePairs = false;  // many-row GEMMs on CTA pairs (tc_gemmp2_kernel) where they fill the GPU
+constexpr bool kUsePairs = true;   // many-row GEMMs on CTA pairs (tc_gemmp2_kernel) where they fill the GPU
 using Big = TcShape<kBN, 2, kStages>;
 using Small = TcShape<kBN, 1, kStages>;
 
