@@ -14,7 +14,7 @@
 // TMA chunk loads as the mma.sync kernel).  Per chunk i:
 //   S_i = Q K_i^T         tcgen05.mma M = 128, N = 64, K = 128 (both operands K-major), into one of two
 //                         64-column TMEM buffers, issued before the softmax of chunk i - 1 has finished;
-//   softmax (4 warps, one query vector per thread): S_i from TMEM, masked and scaled to base 2, online
+//   softmax (8 warps, two threads per query vector): S_i from TMEM, masked and scaled to base 2, online
 //                         max / denominator; P_i = 2^(s - m) rounded to bf16 into shared memory (one
 //                         buffer: the softmax of chunk i writes it only after P_{i-1} V_{i-1} completed);
 //   O += P_i V_i          tcgen05.mma M = 128, N = 128, K = 64, V taken MN-major straight from the page
@@ -23,7 +23,8 @@
 // weights); O and the denominator are then rescaled in TMEM.  Between raises, weights up to 2^8 are
 // summed exactly as the plain online softmax would sum them after its rescale, so the result is the same
 // softmax.  Warp roles: warp 0 lane 0 issues the TMA copies, warp 1 owns TMEM and its lane 0 issues the
-// MMAs, warps 2..5 run the softmax and the output.
+// MMAs, warps 2..9 run the softmax and the output, two threads per query vector (one per half of the keys
+// of a chunk and of the output columns).
 //
 // Importance: the block chunk's scaled scores stay in registers until the final m and denominator are
 // known; the probabilities of the block keys are then summed over the tile's query vectors per key in
@@ -57,6 +58,11 @@ constexpr int kT5Smem = 2 * kT5QHalf + kT5Stages * kStageBytes + kT5PBytes + 102
 constexpr uint32_t kT5TmemCols = 256;             // S (two 64-column buffers) + O (128 columns)
 constexpr uint32_t kT5OCol = 128;                 // first TMEM column of O
 constexpr float kT5Raise = 8.f;                   // base-2 headroom before the running max is raised
+constexpr int kT5SoftWarps = 8;                   // softmax warps: two threads per query vector
+constexpr int kT5Threads = 64 + 32 * kT5SoftWarps;  // + the TMA warp and the MMA warp
+
+// The softmax warps' own barrier (named barrier 1, all 256 of their threads).
+__device__ __forceinline__ void named_sync_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // 3-D TMA load (q rows: d, head, row).
 __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* bar, void* dst, int x, int y, int z) {
@@ -97,7 +103,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t addr, uint32_t l
 }
 
 template <bool FULL>
-__global__ void __launch_bounds__(192, 1) attention_t5_kernel(const __grid_constant__ CUtensorMap pool_map,
+__global__ void __launch_bounds__(kT5Threads, 1) attention_t5_kernel(const __grid_constant__ CUtensorMap pool_map,
                                                               const __grid_constant__ CUtensorMap ibc_map,
                                                               const __grid_constant__ CUtensorMap q_map, AttnArgs a,
                                                               int q_tiles) {
@@ -116,6 +122,8 @@ __global__ void __launch_bounds__(192, 1) attention_t5_kernel(const __grid_const
     __shared__ __align__(8) uint64_t done_bar;
     __shared__ uint64_t valid_s[kT5Stages];
     __shared__ int32_t pt_s[kPtCache];
+    __shared__ float xm_s[2][2][kT5Q];   // per chunk parity and column half: the half-row maxima
+    __shared__ float lx_s[2][kT5Q];      // per column half: the row's partial denominators
     __shared__ uint32_t tmem_slot;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -143,8 +151,8 @@ __global__ void __launch_bounds__(192, 1) attention_t5_kernel(const __grid_const
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&s_free[b], 4);  // one arrival per softmax warp
-            mbar_init(&p_full[b], 4);
+            mbar_init(&s_free[b], kT5SoftWarps);  // one arrival per softmax warp
+            mbar_init(&p_full[b], kT5SoftWarps);
         }
         mbar_init(&pv_bar, 1);
         mbar_init(&done_bar, 1);
@@ -243,45 +251,47 @@ __global__ void __launch_bounds__(192, 1) attention_t5_kernel(const __grid_const
             }
             __syncwarp();
         } else {
-            // ---- softmax and output: one query vector per thread
-            const int quarter = warp & 3;
+            // ---- softmax and output: eight warps, two threads per query vector (each thread owns one half of
+            // the 64 keys of a chunk and one half of the 128 output columns).  Warps 2..9: TMEM lane quarter
+            // warp % 4 (the query vectors 32 (warp % 4) .. + 31), column half (warp - 2) / 4.  The two halves
+            // of a row exchange their chunk maxima through shared memory behind a named barrier; every softmax
+            // warp passes that barrier once per chunk even after one of its waits gave up (it then only
+            // skips its tensor-memory work), so no warp is left waiting there.
+            const int quarter = warp & 3, half = (warp - 2) >> 2;
             const int t = quarter * 32 + lane;                   // query vector within the tile
             const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
             const float sl2 = rsqrtf((float)kD) * 1.4426950408889634f;  // 1/sqrt(d) * log2(e)
             float m_used = -CUDART_INF_F, l = 0.f;
-            float sb[kChunk];                                    // block chunk: scaled scores (importance)
+            float sb[32];                                        // block chunk: this half's scaled scores
             bool alive = true;
             for (int i = 0; i < n_chunks; ++i) {
                 const int st = i % kT5Stages, sbuf = i & 1;
-                bool ok = mbar_wait(&s_full[sbuf], (uint32_t)(i >> 1) & 1u, a.err) &&
+                bool ok = alive && mbar_wait(&s_full[sbuf], (uint32_t)(i >> 1) & 1u, a.err) &&
                           mbar_wait(&kv_full[st], (uint32_t)(i / kT5Stages) & 1u, a.err);  // valid_s is written
-                if (!__all_sync(0xffffffffu, ok)) {
-                    alive = false;
-                    break;
-                }
-                tc_fence_after();
-                float s[kChunk];
-                tmem_ld32(trow + (uint32_t)(sbuf * 64), *reinterpret_cast<float(*)[32]>(s));
-                tmem_ld32(trow + (uint32_t)(sbuf * 64 + 32), *reinterpret_cast<float(*)[32]>(s + 32));
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_free[sbuf]);
-                const uint64_t vmask = valid_s[st];
-                float cmax = -CUDART_INF_F;
-#pragma unroll
-                for (int c = 0; c < kChunk; ++c) {
-                    s[c] = ((vmask >> c) & 1ull) ? s[c] * sl2 : -CUDART_INF_F;
-                    cmax = fmaxf(cmax, s[c]);
-                }
-                // P V of the previous chunk has completed: O is stable and P buffer i % 2 is free
-                if (i >= 1) {
-                    ok = mbar_wait(&pv_bar, (uint32_t)(i - 1) & 1u, a.err);
-                    if (!__all_sync(0xffffffffu, ok)) {
-                        alive = false;
-                        break;
-                    }
+                alive = __all_sync(0xffffffffu, ok);
+                float s[32];
+                float cm = -CUDART_INF_F;
+                const uint32_t vm = (uint32_t)(valid_s[st] >> (32 * half));
+                if (alive) {
                     tc_fence_after();
+                    tmem_ld32(trow + (uint32_t)(sbuf * 64 + half * 32), s);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s_free[sbuf]);
+                    if (vm != 0xffffffffu) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) s[c] = ((vm >> c) & 1u) ? s[c] : -CUDART_INF_F;
+                    }
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) cm = fmaxf(cm, s[c]);
                 }
+                xm_s[sbuf][half][t] = cm == -CUDART_INF_F ? cm : cm * sl2;
+                named_sync_softmax();
+                const float cmax = fmaxf(xm_s[sbuf][0][t], xm_s[sbuf][1][t]);  // the same value in both halves
+                // P V of the previous chunk has completed: O is stable and the P buffer is free
+                if (alive && i >= 1) alive = __all_sync(0xffffffffu, mbar_wait(&pv_bar, (uint32_t)(i - 1) & 1u, a.err));
+                if (!alive) continue;
+                tc_fence_after();
                 // raise the running max only by more than kT5Raise; O and the denominator follow it
                 float f = 1.f;
                 if (m_used == -CUDART_INF_F) {
@@ -293,20 +303,20 @@ __global__ void __launch_bounds__(192, 1) attention_t5_kernel(const __grid_const
                 }
                 if (__any_sync(0xffffffffu, f != 1.f)) {  // TMEM access is warp-collective: factor 1 elsewhere
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kD; c0 += 32) {
+                    for (int c0 = 0; c0 < kD / 2; c0 += 32) {
                         float v[32];
-                        tmem_ld32(trow + kT5OCol + (uint32_t)c0, v);
+                        tmem_ld32(trow + kT5OCol + (uint32_t)(half * 64 + c0), v);
 #pragma unroll
                         for (int c = 0; c < 32; ++c) v[c] *= f;
-                        tmem_st32(trow + kT5OCol + (uint32_t)c0, v);
+                        tmem_st32(trow + kT5OCol + (uint32_t)(half * 64 + c0), v);
                     }
                 }
                 const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;
                 float rs = 0.f;
-                uint32_t pk[kChunk / 2];
+                uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < kChunk; c += 2) {
-                    const float p0 = exp2f(s[c] - mu), p1 = exp2f(s[c + 1] - mu);
+                for (int c = 0; c < 32; c += 2) {
+                    const float p0 = exp2f(fmaf(s[c], sl2, -mu)), p1 = exp2f(fmaf(s[c + 1], sl2, -mu));
                     rs += p0 + p1;
                     __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
                     pk[c / 2] = *reinterpret_cast<uint32_t*>(&b2);
@@ -314,18 +324,19 @@ __global__ void __launch_bounds__(192, 1) attention_t5_kernel(const __grid_const
                 l += rs;
                 if (FULL && i == n_chunks - 1) {
 #pragma unroll
-                    for (int c = 0; c < kChunk; ++c) sb[c] = s[c];
+                    for (int c = 0; c < 32; ++c) sb[c] = s[c] == -CUDART_INF_F ? s[c] : s[c] * sl2;
                 }
-                // P row t: 128 bytes, 16-byte chunk c at (c ^ (t & 7)) (the 128-byte swizzle)
+                // P row t: 128 bytes, 16-byte chunk cc at (cc ^ (t & 7)) (the 128-byte swizzle); this half writes
+                // chunks 4 half .. 4 half + 3
                 uint8_t* prow = p_s + (t >> 3) * 1024 + (t & 7) * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4*>(prow + ((c ^ (t & 7)) << 4)) =
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (t & 7)) << 4)) =
                         make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                 // V rows of keys the copies left unfilled may hold stale bits: P is 0 there, so make V 0 too
-                if (vmask != ~0ull) {
+                if (half == 0 && valid_s[st] != ~0ull) {
                     const int r = t & 63, h = t >> 6;
-                    if (!((vmask >> r) & 1ull)) {
+                    if (!((valid_s[st] >> r) & 1ull)) {
                         uint4* vr = reinterpret_cast<uint4*>(kv_s + st * kStageBytes + 2 * kHalf + h * kHalf + r * 128);
 #pragma unroll
                         for (int c = 0; c < 8; ++c) vr[c] = make_uint4(0, 0, 0, 0);
@@ -336,19 +347,22 @@ __global__ void __launch_bounds__(192, 1) attention_t5_kernel(const __grid_const
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_full[sbuf]);
             }
-            // the last P V has completed: normalise and write this thread's query vector
+            // the last P V has completed: normalise and write this thread's half of the query vector
             if (alive) alive = __all_sync(0xffffffffu, mbar_wait(&pv_bar, (uint32_t)(n_chunks - 1) & 1u, a.err));
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            lx_s[half][t] = l;
+            named_sync_softmax();
+            const float lt = lx_s[0][t] + lx_s[1][t];            // fixed order: the same in both halves
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
             const bool live = t < u.nq;
             if (alive) {
                 tc_fence_after();
                 const int qi = u.q0 + t;
                 const int row = qi / G, hh = u.g * G + (qi - row * G);
-                bf16* dst = reinterpret_cast<bf16*>(a.o) + ((size_t)(u.row_base + row) * a.Hq + hh) * kD;
+                bf16* dst = reinterpret_cast<bf16*>(a.o) + ((size_t)(u.row_base + row) * a.Hq + hh) * kD + half * 64;
 #pragma unroll 1
-                for (int c0 = 0; c0 < kD; c0 += 32) {
+                for (int c0 = 0; c0 < kD / 2; c0 += 32) {
                     float v[32];
-                    tmem_ld32(trow + kT5OCol + (uint32_t)c0, v);
+                    tmem_ld32(trow + kT5OCol + (uint32_t)(half * 64 + c0), v);
                     if (live) {
 #pragma unroll
                         for (int c = 0; c < 32; c += 8) {
@@ -372,14 +386,15 @@ __global__ void __launch_bounds__(192, 1) attention_t5_kernel(const __grid_const
                     float* colbuf = reinterpret_cast<float*>(kv_s);  // [128 query vectors][65]
                     const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;
 #pragma unroll
-                    for (int c = 0; c < kChunk; ++c)
-                        colbuf[t * 65 + c] =
-                            (alive && live && sb[c] != -CUDART_INF_F && l > 0.f) ? exp2f(sb[c] - mu) * inv : 0.f;
-                    tc::named_sync_epilogue();
-                    if (t < a.B) {
+                    for (int c = 0; c < 32; ++c)
+                        colbuf[t * 65 + half * 32 + c] =
+                            (alive && live && sb[c] != -CUDART_INF_F && lt > 0.f) ? exp2f(sb[c] - mu) * inv : 0.f;
+                    named_sync_softmax();
+                    const int j = half * 128 + t;
+                    if (j < a.B) {
                         float col = 0.f;
-                        for (int r = 0; r < kT5Q; ++r) col += colbuf[r * 65 + t];
-                        a.imp_part[(size_t)unit * a.B + t] = col;
+                        for (int r = 0; r < kT5Q; ++r) col += colbuf[r * 65 + j];
+                        a.imp_part[(size_t)unit * a.B + j] = col;
                     }
                 }
             }
@@ -444,9 +459,9 @@ int launch_attention_t5(const AttnArgs& a, int q_tiles, cudaStream_t s) {
     if (!make_q_map(&q_map, a.q, a.q_rows_cap, a.Hq, G)) return -1;
     const dim3 grid(a.N, a.Hkv, q_tiles);
     if (a.row_offsets == nullptr)
-        return launched(launch_pdl(attention_t5_kernel<true>, grid, dim3(192), kT5Smem, s, 0, pool_map, ibc_map, q_map, a,
+        return launched(launch_pdl(attention_t5_kernel<true>, grid, dim3(kT5Threads), kT5Smem, s, 0, pool_map, ibc_map, q_map, a,
                                    q_tiles));
-    return launched(launch_pdl(attention_t5_kernel<false>, grid, dim3(192), kT5Smem, s, 0, pool_map, ibc_map, q_map, a,
+    return launched(launch_pdl(attention_t5_kernel<false>, grid, dim3(kT5Threads), kT5Smem, s, 0, pool_map, ibc_map, q_map, a,
                                q_tiles));
 }
 
