@@ -22,6 +22,7 @@ import dataclasses
 import datetime
 import hashlib
 import json
+import math
 import os
 import re
 import statistics
@@ -194,7 +195,8 @@ def step_work(case: fs.Case, R: int, kept_per_req, plen):
     the kept rows;
     layers 2..L-1 on the R kept rows (QKV, ragged attention, O, norm, gate/up, down, norm); LM head;
     combine + decode.  Norms read the float32 residual and write bf16 rows (the gathering norm also
-    writes the compacted float32 rows)."""
+    writes the compacted float32 rows).  With more than 256 kept-row slots (N x k_max, bf16) every
+    kept-row GEMM is two launches, of which the one whose range misses the live row count does no work."""
     s = case.shape
     L, D = s.n_layers, s.hidden
     N, B = case.work.n_requests, case.work.block
@@ -215,9 +217,18 @@ def step_work(case: fs.Case, R: int, kept_per_req, plen):
     for kc in ("gemm_qkv", "attn_ragged", "gemm_o", "gemm_gateup", "gemm_down"):
         by, fl = algorithmic_work(kc, case, R, kept_per_req, plen)
         work.append((kc, n_kept_layers, by, fl))
+    w = case.work
+    k_cap = (min(B, math.ceil(w.forced_keep_frac * B)) if w.forced_keep_frac is not None and w.forced_keep_frac >= 0
+             else w.k_max)
     work.append(("row_norm", 2 * n_kept_layers, R * D * (4 + e), 0.0))
     by, fl = algorithmic_work("gemm_lmhead", case, R, kept_per_req, plen)
     work.append(("gemm_lmhead", 1, by, fl))
+    if s.dtype == "bf16" and N * k_cap > 256:
+        # kept-row bound above 256: each kept-row GEMM is a few-row and a many-row launch, and the one whose
+        # range the live row count misses exits after its wait (no work)
+        for kc in ("gemm_qkv", "gemm_o", "gemm_gateup", "gemm_down"):
+            work.append((kc, n_kept_layers, 0.0, 0.0))
+        work.append(("gemm_lmhead", 1, 0.0, 0.0))
     work.append(("decode", 2, R * ((s.vocab + 127) // 128) * 12 + 3 * N * B * 4, 0.0))
     return work
 
@@ -281,8 +292,9 @@ def family_rooflines(per_class: dict, work, peaks: dict) -> dict:
 def source_digest(kclass: str) -> str:
     """Digest of the sources that build a kernel class (recorded traffic is used only while it matches)."""
     shared = ["common.cuh", "launch.h"]
-    files = {"gemm": ["tc_gemm.cu", "tc_gemm_kernel.cuh", "gemm_simt.cu"],
-             "attn": ["attention_tc.cu", "attention.cu", "tc_gemm_kernel.cuh"], "row": ["rows.cu"],
+    files = {"gemm": ["tc_gemm.cu", "tc_gemm_kernel.cuh", "tc_gemm_persist.cuh", "gemm_simt.cu"],
+             "attn": ["attention_tc.cu", "attention_t5.cu", "attention_pages.cuh", "attention.cu",
+                      "tc_gemm_kernel.cuh"], "row": ["rows.cu"],
              "qkv": ["rows.cu"], "embed": ["rows.cu"], "select": ["select.cu"], "decode": ["decode.cu"]}
     key = kclass.split("_")[0]
     h = hashlib.sha256()

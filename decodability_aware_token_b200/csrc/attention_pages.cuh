@@ -74,5 +74,28 @@ __device__ __forceinline__ uint64_t issue_chunk(const AttnArgs& a, const Unit& u
     return mask;
 }
 
+// Ask L2 for the K and V rows of prefix chunk `ci` (one bulk prefetch per page and K / V; no shared memory,
+// no barrier), issued one chunk ahead of the ring's copies: one more chunk of DRAM requests in flight per CTA
+// than the shared-memory ring holds, with an L2 footprint (one chunk per CTA, ~10 MB) far below its capacity.
+// (Four chunks ahead raised DRAM reads by a fifth: the lines were evicted before their copies came.)
+// Pages past the prefix or with an out-of-range id are skipped; the block chunk is not prefetched.
+__device__ __forceinline__ void prefetch_chunk_l2(const AttnArgs& a, const Unit& u, int ci, int n_prefix_chunks,
+                                                  const int32_t* pt) {
+    if (ci >= n_prefix_chunks) return;
+    const int S = a.page_size;
+    const uint32_t bytes = (uint32_t)S * kD * 2;  // S rows of 256 bytes: a multiple of 16
+    for (int p = 0; p < kChunk / S; ++p) {
+        const int t0 = ci * kChunk + p * S;
+        if (t0 >= u.P) break;
+        const int page = pt[t0 / S];
+        if (page < 0 || page >= a.n_pages) continue;
+        const size_t krow = ((((size_t)page * a.L + a.layer) * 2 + 0) * a.Hkv + u.g) * (size_t)S;
+        const uint8_t* kp = reinterpret_cast<const uint8_t*>(a.kv_pool) + krow * kD * 2;
+        const uint8_t* vp = kp + (size_t)a.Hkv * S * kD * 2;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kp), "r"(bytes) : "memory");
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(vp), "r"(bytes) : "memory");
+    }
+}
+
 }  // namespace
 }  // namespace focus

@@ -165,7 +165,12 @@ struct GemmArgs {
     const float2* rope_tab;     // tensor-core epilogues: [positions][d / 2] (cos, sin) of pos * inv_freq
     int max_prefix, block, n_layers, layer, Hq, Hkv;
     int* err;
+    // Row bounds above 256 with a live count known only on the device: the few-row and the many-row kernel
+    // are both launched, and each works only if the live count is in its range (else it exits after its
+    // programmatic-launch wait).  0: no gate, 1: live <= 256 only (few-row kernel), 2: live > 256 only.
+    int live_gate;
 };
+constexpr int kGateFewRows = 1, kGateManyRows = 2;
 template <typename T> int launch_gemm_simt(Epi epi, const GemmArgs& g, cudaStream_t s);
 constexpr int kSimtTileN = 64;
 

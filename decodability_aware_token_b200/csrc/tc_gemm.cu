@@ -39,7 +39,7 @@ using namespace tc;
 // swapped kernel.  More kept rows than that (large batches) take the row-major kernel, whose CTAs with
 // all rows beyond the live row count exit after the wait.
 constexpr int kBN = 128, kStages = 4;
-constexpr int kSmallRows = 256;  // GEMMs with at most this many rows run on the swapped kernel
+constexpr int kSmallRows = kTcFewRows;  // GEMMs with at most this many rows run on the swapped kernel
 constexpr bool kUsePairs = true;   // many-row GEMMs on CTA pairs (tc_gemmp2_kernel) where they fill the GPU
 using Big = TcShape<kBN, 2, kStages>;
 using Small = TcShape<kBN, 1, kStages>;
@@ -55,10 +55,14 @@ struct TcPlan {
     CUtensorMap map_h32, map_o32, map_act32;  // 32-row boxes: token operand of the swapped kernel
     std::unordered_map<const void*, CUtensorMap> wmap;   // weight pointer -> map (box rows = tile N or N/2)
     std::unordered_map<const void*, CUtensorMap> wmap2;  // the same with 256-row boxes (128 for gate / up)
+    std::unordered_map<const void*, CUtensorMap> wmap32; // O and down weights in 32-row boxes (column slabs)
     int* err;
     int sms;
     int max_clusters[kTMaxSplits + 1];  // co-resident clusters of the swapped kernel with s CTAs (0: not launchable)
     int max_pairs;                      // co-resident CTA pairs of the paired persistent kernel (0: not used)
+    // fp32 maps of the residual streams and the split-tile partial buffer (pointer -> rows, map), built on
+    // first use: the residual epilogue adds and stores through them
+    std::unordered_map<const void*, std::pair<uint64_t, CUtensorMap>> fmap;
 };
 
 
@@ -106,6 +110,10 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
         p->wmap2[w.wup[l]] = m;
         ok = ok && make_map(&m, w.wdown[l], dm.D, dm.F, 2 * kBN);
         p->wmap2[w.wdown[l]] = m;
+        ok = ok && make_map(&m, w.wo[l], dm.D, HD, 32);
+        p->wmap32[w.wo[l]] = m;
+        ok = ok && make_map(&m, w.wdown[l], dm.D, dm.F, 32);
+        p->wmap32[w.wdown[l]] = m;
     }
     CUtensorMap m;
     ok = ok && make_map(&m, w.lm_head, dm.V, dm.D, kBN);
@@ -132,11 +140,11 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
          set_smem((const void*)tc_gemmt_kernel<EPI_LMHEAD>, kTSmem) &&
          set_smem((const void*)tc_gemmp_kernel<256, EPI_SWIGLU>, PShape<256>::SMEM) &&
          set_smem((const void*)tc_gemmp_kernel<256, EPI_LMHEAD>, PShape<256>::SMEM) &&
-         set_smem((const void*)tc_gemmp_kernel<256, EPI_RESID>, PShape<256>::SMEM) &&
+         set_smem((const void*)tc_gemmp_kernel<256, EPI_RESID>, PShape<256>::SMEM_RESID) &&
          set_smem((const void*)tc_gemmp_kernel<256, EPI_QKV>, PShape<256>::SMEM) &&
          set_smem((const void*)tc_gemmp_kernel<128, EPI_SWIGLU>, PShape<128>::SMEM) &&
          set_smem((const void*)tc_gemmp_kernel<128, EPI_LMHEAD>, PShape<128>::SMEM) &&
-         set_smem((const void*)tc_gemmp_kernel<128, EPI_RESID>, PShape<128>::SMEM) &&
+         set_smem((const void*)tc_gemmp_kernel<128, EPI_RESID>, PShape<128>::SMEM_RESID) &&
          set_smem((const void*)tc_gemmp_kernel<128, EPI_QKV>, PShape<128>::SMEM) &&
          set_smem((const void*)tc_gemmp2_kernel<EPI_SWIGLU>, kP2Smem) &&
          set_smem((const void*)tc_gemmp2_kernel<EPI_LMHEAD>, kP2Smem) &&
@@ -203,6 +211,24 @@ int tc_lm_tiles(const TcPlan* p) { return p ? (p->dm.V + kBN - 1) / kBN : 0; }
 
 namespace {
 
+// fp32 [rows, cols] map of `base` (cached per pointer; rebuilt when the row count changes); null on failure
+const CUtensorMap* f32_map(TcPlan* p, const void* base, uint64_t rows, uint64_t cols) {
+    auto it = p->fmap.find(base);
+    if (it != p->fmap.end() && it->second.first == rows) return &it->second.second;
+    CUtensorMap m;
+    if (!make_map_f32(&m, base, rows, cols)) return nullptr;
+    auto& slot = p->fmap[base];
+    slot = {rows, m};
+    return &slot.second;
+}
+
+// Slabs per tile when a residual GEMM has fewer pair tiles than co-resident pairs (then all its tiles form
+// one partial round): 4 or 2 if that many slabs of every tile still fit on the pairs.
+int launch_slabs(Epi epi, long long tiles, int max_pairs) {
+    if (epi != EPI_RESID || tiles >= max_pairs) return 1;
+    return tiles * 4 <= max_pairs ? 4 : tiles * 2 <= max_pairs ? 2 : 1;
+}
+
 // Swapped GEMM: 128-feature tiles x all live tokens, split K over a cluster of 1..8 CTAs (each slice keeps
 // at least one K block).  The LM head (many feature tiles) does not split.
 int tc_gemm_swapped(TcPlan* p, Epi epi, GemmArgs g, cudaStream_t s) {
@@ -247,13 +273,17 @@ int tc_gemm_persistent(TcPlan* p, Epi epi, GemmArgs g, int tiles, cudaStream_t s
         g.n_tiles = (g.N + kBN - 1) / kBN;  // statistics per 128 vocabulary columns, as the combine reads them
         g.tile_n = kBN;
     }
+    const CUtensorMap* c = a;  // the residual stream (EPI_RESID), unused otherwise
+    if (epi == EPI_RESID && !(c = f32_map(p, g.resid, (uint64_t)g.M_bound, (uint64_t)g.N))) return -1;
     const dim3 grid(tiles < p->sms ? tiles : p->sms, 1, 1), blk(192);
     const int smem = PShape<BN>::SMEM;
     switch (epi) {
-        case EPI_SWIGLU: return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_SWIGLU>, grid, blk, smem, s, 0, *a, *b, *b2, g, p->err));
-        case EPI_LMHEAD: return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_LMHEAD>, grid, blk, smem, s, 0, *a, *b, *b2, g, p->err));
-        case EPI_RESID: return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_RESID>, grid, blk, smem, s, 0, *a, *b, *b2, g, p->err));
-        case EPI_QKV: return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_QKV>, grid, blk, smem, s, 0, *a, *b, *b2, g, p->err));
+        case EPI_SWIGLU: return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_SWIGLU>, grid, blk, smem, s, 0, *a, *b, *b2, *c, g, p->err));
+        case EPI_LMHEAD: return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_LMHEAD>, grid, blk, smem, s, 0, *a, *b, *b2, *c, g, p->err));
+        case EPI_RESID:
+            return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_RESID>, grid, blk, PShape<BN>::SMEM_RESID, s, 0, *a, *b, *b2,
+                                       *c, g, p->err));
+        case EPI_QKV: return launched(launch_pdl(tc_gemmp_kernel<BN, EPI_QKV>, grid, blk, smem, s, 0, *a, *b, *b2, *c, g, p->err));
         default: return -1;
     }
 }
@@ -275,15 +305,39 @@ int tc_gemm_pairs(TcPlan* p, Epi epi, GemmArgs g, int tiles, cudaStream_t s) {
         g.n_tiles = (g.N + kBN - 1) / kBN;
         g.tile_n = kBN;
     }
-    const int pairs = tiles < p->max_pairs ? tiles : p->max_pairs;
+    // EPI_RESID: the residual stream, and the weights in 32-row boxes for the column slabs of a last round
+    const CUtensorMap *c = a, *bt = a;
+    if (epi == EPI_RESID) {
+        if (!(c = f32_map(p, g.resid, (uint64_t)g.M_bound, (uint64_t)g.N))) return -1;
+        auto it = p->wmap32.find(g.B);
+        if (it == p->wmap32.end()) return -1;
+        bt = &it->second;
+    }
+    // fewer tiles than pairs: enough pairs for the column slabs of every tile
+    const int pairs = tiles < p->max_pairs ? tiles * launch_slabs(epi, tiles, p->max_pairs) : p->max_pairs;
     const dim3 grid(2 * pairs, 1, 1), blk(192);
     switch (epi) {
-        case EPI_SWIGLU: return launched(launch_pdl(tc_gemmp2_kernel<EPI_SWIGLU>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, g, p->err));
-        case EPI_LMHEAD: return launched(launch_pdl(tc_gemmp2_kernel<EPI_LMHEAD>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, g, p->err));
-        case EPI_RESID: return launched(launch_pdl(tc_gemmp2_kernel<EPI_RESID>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, g, p->err));
-        case EPI_QKV: return launched(launch_pdl(tc_gemmp2_kernel<EPI_QKV>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, g, p->err));
+        case EPI_SWIGLU: return launched(launch_pdl(tc_gemmp2_kernel<EPI_SWIGLU>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, *c, *bt, g, p->err));
+        case EPI_LMHEAD: return launched(launch_pdl(tc_gemmp2_kernel<EPI_LMHEAD>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, *c, *bt, g, p->err));
+        case EPI_RESID: return launched(launch_pdl(tc_gemmp2_kernel<EPI_RESID>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, *c, *bt, g, p->err));
+        case EPI_QKV: return launched(launch_pdl(tc_gemmp2_kernel<EPI_QKV>, grid, blk, kP2Smem, s, 2, *a, *b, *b2, *c, *bt, g, p->err));
         default: return -1;
     }
+}
+
+// Column slabs per tile of a last partial round of `tiles` pair tiles over `pairs` pairs (residual GEMMs:
+// the most of 4 or 2 that keeps that round within the pairs; the kernel applies the same rule).
+int slabs(Epi epi, long long tiles, int pairs) {
+    const long long rem = tiles % pairs;
+    if (epi != EPI_RESID || rem == 0) return 1;
+    return rem * 4 <= pairs ? 4 : rem * 2 <= pairs ? 2 : 1;
+}
+
+// Rounds of tile-MMA time a pair launch takes: the full rounds, plus a slab's share of a round for the last.
+double pair_rounds(Epi epi, long long tiles, int max_pairs) {
+    const int pairs = (int)(tiles < max_pairs ? tiles * launch_slabs(epi, tiles, max_pairs) : max_pairs);
+    const long long full = tiles / pairs, rem = tiles % pairs;
+    return (double)full + (rem ? 1.0 / slabs(epi, tiles, pairs) : 0.0);
 }
 
 // Column tiles of width bn (0 if the epilogue needs whole tiles and N does not divide).
@@ -295,11 +349,10 @@ int persist_col_tiles(Epi epi, int N, int bn) {
 
 }  // namespace
 
-int tc_gemm(TcPlan* p, Epi epi, const GemmArgs& g0, cudaStream_t s) {
-    if (g0.M_bound <= 0) return 0;
-    if (epi == EPI_PARTIAL) return -1;  // partial sums are the CUDA-core path's; these kernels fuse their epilogues
-    GemmArgs g = g0;
-    if (g.M_bound <= kSmallRows) return tc_gemm_swapped(p, epi, g, s);
+namespace {
+
+// GEMMs of more than kSmallRows rows (at the row bound)
+int tc_gemm_many(TcPlan* p, Epi epi, GemmArgs g, cudaStream_t s) {
     {
         // Persistent kernel when there are enough tiles to fill the SMs.  Of 256- and 128-wide tiles take the
         // one with the shorter expected time: full waves of tiles (at the row bound) x tile width, a 128-wide
@@ -311,10 +364,12 @@ int tc_gemm(TcPlan* p, Epi epi, const GemmArgs& g0, cudaStream_t s) {
         const double c128 = n128 ? (double)((t128 + p->sms - 1) / p->sms) * 128.0 * 1.15 : 1e30;
         if (p->max_pairs > 0 && n256) {
             // pairs: 256 x 256 tiles, one round = max_pairs tiles; a round takes about as long as a round of
-            // 128 x 256 tiles on single CTAs, at two thirds of their operand bytes per flop
+            // 128 x 256 tiles on single CTAs, at two thirds of their operand bytes per flop.  Residual GEMMs cut
+            // the tiles of a last partial round into 64- or 128-column slabs (pair_rounds).
             const long long tp = (long long)((g.M_bound + 255) / 256) * n256;
-            const double cp = (double)((tp + p->max_pairs - 1) / p->max_pairs) * 256.0 * (2.0 * p->max_pairs / p->sms);
-            if (tp >= p->max_pairs && cp <= c256 && cp <= c128) return tc_gemm_pairs(p, epi, g, (int)tp, s);
+            const double cp = pair_rounds(epi, tp, p->max_pairs) * 256.0 * (2.0 * p->max_pairs / p->sms);
+            if ((tp >= p->max_pairs || epi == EPI_RESID) && cp <= c256 && cp <= c128)
+                return tc_gemm_pairs(p, epi, g, (int)tp, s);
         }
         if (n256 && t256 >= p->sms && c256 <= c128) return tc_gemm_persistent<256>(p, epi, g, (int)t256, s);
         if (n128 && t128 >= p->sms) return tc_gemm_persistent<128>(p, epi, g, (int)t128, s);
@@ -357,6 +412,25 @@ int tc_gemm(TcPlan* p, Epi epi, const GemmArgs& g0, cudaStream_t s) {
         default:
             return -1;
     }
+}
+
+}  // namespace
+
+int tc_gemm(TcPlan* p, Epi epi, const GemmArgs& g0, cudaStream_t s) {
+    if (g0.M_bound <= 0) return 0;
+    if (epi == EPI_PARTIAL) return -1;  // partial sums are the CUDA-core path's; these kernels fuse their epilogues
+    GemmArgs g = g0;
+    if (g.M_bound <= kSmallRows) return tc_gemm_swapped(p, epi, g, s);
+    if (g.M_dev == nullptr) return tc_gemm_many(p, epi, g, s);
+    // kept rows whose bound exceeds the few-row kernel but whose live count may not: launch both kernels;
+    // each reads the live count after its programmatic wait and only one of them works
+    GemmArgs gf = g;
+    gf.live_gate = kGateFewRows;
+    const int n_few = tc_gemm_swapped(p, epi, gf, s);
+    if (n_few < 0) return -1;
+    g.live_gate = kGateManyRows;
+    const int n_many = tc_gemm_many(p, epi, g, s);
+    return n_many < 0 ? -1 : n_few + n_many;
 }
 
 }  // namespace focus

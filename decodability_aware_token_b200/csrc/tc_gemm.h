@@ -23,5 +23,7 @@ int tc_plan_create(TcPlan** out, const Dims& dm, const TcWeights& w, void* h, vo
 void tc_plan_destroy(TcPlan* p);
 int tc_lm_tiles(const TcPlan* p);
 int tc_gemm(TcPlan* p, Epi epi, const GemmArgs& g, cudaStream_t s);
+// GEMMs of at most this many rows run on the swapped few-row kernel
+constexpr int kTcFewRows = 256;
 
 }  // namespace focus

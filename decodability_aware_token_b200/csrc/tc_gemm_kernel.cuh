@@ -191,7 +191,9 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
     const int kb0 = (int)((long long)nk_all * split / splits);
     const int kb1 = (int)((long long)nk_all * (split + 1) / splits);
     const int nk = kb1 - kb0;
-    const int n_pre = min(nk, STAGES);  // stages whose weight tiles go out before the programmatic wait
+    // stages whose weight tiles go out before the programmatic wait (none when the few-row kernel may take
+    // this launch: the copies would be wasted there)
+    const int n_pre = g.live_gate == kGateManyRows ? 0 : min(nk, STAGES);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -232,7 +234,9 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
     }
     pdl_wait();
 
-    const int M = g.M_dev ? *g.M_dev : g.M_bound;
+    const int M = g.live_gate == kGateManyRows && (g.M_dev ? *g.M_dev : g.M_bound) <= 256
+                      ? 0  // the few-row kernel's launch
+                      : (g.M_dev ? *g.M_dev : g.M_bound);
     if (m0 >= M) {  // whole CTA: let the early weight copies land, release TMEM, leave
         if (warp == 0 && lane == 0)
             for (int s = 0; s < n_pre; ++s) {
@@ -510,7 +514,8 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
     // output features of the tile: 128 (QKV: one head; residual GEMMs; LM head), or 64 gate + 64 up (SwiGLU)
     const int fbase = EPI == EPI_SWIGLU ? n_tile * 64 : n_tile * 128;
     // stages whose weight tiles go out before the wait: as many as the ring holds at the token bound
-    const int n_pre = min(nk, min(kTMaxStages, kTRing / (kTW + xb_bound * kTXBox)));
+    // (none when the many-row kernel may take this launch: the copies would be wasted there)
+    const int n_pre = g.live_gate == kGateFewRows ? 0 : min(nk, min(kTMaxStages, kTRing / (kTW + xb_bound * kTXBox)));
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < kTMaxStages; ++st) {
@@ -543,7 +548,8 @@ __global__ void __launch_bounds__(192, 2) tc_gemmt_kernel(const __grid_constant_
     }
     pdl_wait();
 
-    const int M = min(g.M_dev ? *g.M_dev : Mb, Mb);
+    const int live_rows = g.M_dev ? *g.M_dev : g.M_bound;
+    const int M = g.live_gate == kGateFewRows && live_rows > kTMaxTok ? 0 : min(live_rows, Mb);  // 0: the many-row kernel's
     if (M <= 0) {  // the whole grid: let the early weight copies land, release TMEM, leave
         if (warp == 0 && lane == 0)
             for (int st = 0; st < n_pre; ++st) {
@@ -769,6 +775,21 @@ inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               promote_256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D fp32 row-major [rows, cols] array, box = [32 rows, 32 cols] (128-byte rows), 128-byte swizzle: the
+// staging boxes of the persistent GEMMs' residual epilogue (TMA reductions into the residual stream, TMA
+// stores of split-tile partial sums).
+inline bool make_map_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 4};
+    const cuuint32_t box[2] = {32u, 32u};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

@@ -31,6 +31,7 @@ struct PShape {
     static constexpr int STAGE = A_BYTES + B_BYTES;
     static constexpr int STAGES = (192 * 1024) / STAGE;         // 4 stages at BN = 256, 6 at BN = 128
     static constexpr int SMEM = STAGES * STAGE + 1024;          // + alignment slack
+    static constexpr int SMEM_RESID = SMEM + 32 * 1024;         // + the residual epilogue's staging boxes
     static constexpr uint32_t TMEM_COLS = 2 * BN;               // two accumulators
     static_assert(BN == 128 || BN == 256, "MMA N");
     static_assert(STAGES >= 2 && STAGES <= 8, "ring depth");
@@ -46,6 +47,62 @@ __device__ __forceinline__ void persist_tile(int t, int Mt, int Nt, int Bm, int&
     const int bw = min(Bm, Mt - band * Bm);   // only the last band may be narrower
     n = r / bw;
     m = band * Bm + (r - n * bw);
+}
+
+// ---- residual epilogue through TMA reductions
+// Each epilogue warp moves 32 rows x 32 columns of the accumulator at a time into a 4 KB staging box in
+// shared memory (fp32 rows of 128 bytes with the 128-byte swizzle the tensor map names: 16-byte piece q of
+// row r sits at piece q ^ (r % 8)), and one lane adds the box into the residual stream with a TMA reduction
+// (cp.reduce.async.bulk.tensor, .add on f32).  The residual never enters the SM, every global access is a
+// whole 128-byte line, and each element receives exactly one addition (x + acc, rounded once, as a plain
+// read-modify-write would give).  Rows at or past the live row count add +0; boxes wholly past it are not
+// sent.  Two boxes per warp alternate; a box is rewritten only after the reduction issued from it two boxes
+// earlier has finished reading it.
+constexpr int kResidBox = 32 * 32 * 4;            // one staging box: 4 KB
+constexpr int kResidStage = 4 * 2 * kResidBox;    // four epilogue warps x two boxes: 32 KB
+static_assert(PShape<256>::SMEM_RESID - PShape<256>::SMEM == kResidStage &&
+                  PShape<128>::SMEM_RESID - PShape<128>::SMEM == kResidStage,
+              "staging boxes after the ring");
+static_assert(PShape<256>::SMEM_RESID <= 227 * 1024 && PShape<128>::SMEM_RESID <= 227 * 1024, "one CTA per SM");
+
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int x, int y) {
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(map), "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// at most one bulk group of this thread still reading shared memory
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// every bulk group of this thread complete (its global writes performed)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// `cols` (a multiple of 32) accumulator columns of this warp's 32 TMEM lanes through the staging boxes, added
+// into rows row0 .. row0 + 31, columns col0 .. of the residual stream.  Rows at or past `row_end` add +0 and
+// boxes wholly past it are skipped.  `boxes` = this warp's two staging boxes, `nbox` = boxes this warp has
+// sent so far.
+__device__ __forceinline__ void resid_add_tma(const CUtensorMap* map, uint8_t* boxes, uint32_t tacc, int cols, int row0,
+                                              int col0, int row_end, uint32_t& nbox) {
+    const int lane = threadIdx.x & 31;
+    const bool live = row0 + lane < row_end;
+    const bool any = row0 < row_end;  // warp-uniform
+#pragma unroll 1
+    for (int c0 = 0; c0 < cols; c0 += 32) {
+        float v[32];
+        tmem_ld32(tacc + c0, v);  // warp-collective: every lane
+        if (!any) continue;
+        uint8_t* box = boxes + (nbox & 1u) * kResidBox;
+        if (lane == 0 && nbox >= 2) bulk_wait_read_1();
+        __syncwarp();
+        uint8_t* rowp = box + lane * 128;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(rowp + ((q ^ (lane & 7)) << 4)) =
+                live ? make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the box is visible to the TMA unit
+        __syncwarp();
+        if (lane == 0) tma_reduce_add_2d(map, box, col0 + c0, row0);
+        ++nbox;
+    }
 }
 
 // Epilogue of one accumulator (128 rows x BN columns) for this thread's row; `tacc` is the TMEM address
@@ -182,10 +239,12 @@ __device__ __forceinline__ void persist_epilogue(const GemmArgs& g, uint32_t tac
     }
 }
 
+// tmC: the fp32 residual stream (box 32 columns x 32 rows, 128-byte swizzle), read by EPI_RESID only.
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1) tc_gemmp_kernel(const __grid_constant__ CUtensorMap tmA,
                                                           const __grid_constant__ CUtensorMap tmB,
-                                                          const __grid_constant__ CUtensorMap tmB2, GemmArgs g,
+                                                          const __grid_constant__ CUtensorMap tmB2,
+                                                          const __grid_constant__ CUtensorMap tmC, GemmArgs g,
                                                           int* err) {
     pdl_trigger();
     using S = PShape<BN>;
@@ -228,7 +287,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemmp_kernel(const __grid_constant_
     }
     pdl_wait();
 
-    const int M = min(g.M_dev ? *g.M_dev : g.M_bound, g.M_bound);
+    const int live = min(g.M_dev ? *g.M_dev : g.M_bound, g.M_bound);
+    const int M = g.live_gate == kGateManyRows && live <= 256 ? 0 : live;  // 0: the few-row kernel's launch
     const int Mt = (M + 127) / 128;
     const int Nt = EPI == EPI_SWIGLU ? g.N / (BN / 2) : (g.N + BN - 1) / BN;
     const int T = Mt * Nt;
@@ -310,21 +370,29 @@ __global__ void __launch_bounds__(192, 1) tc_gemmp_kernel(const __grid_constant_
     } else {
         // ---- epilogue: warps 2..5, TMEM lane quarter = warp % 4, one output row per thread
         const int quarter = warp & 3;
+        uint8_t* boxes = smem + S::STAGES * S::STAGE + quarter * 2 * kResidBox;  // EPI_RESID staging
+        uint32_t nbox = 0;
         int it = 0;
+        if (EPI == EPI_RESID && lane == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmC) : "memory");
         for (int t = blockIdx.x; t < T; t += gridDim.x, ++it) {
             const int b = it & 1;
             const uint32_t u = (uint32_t)(it >> 1) & 1u;
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], u, err));
-            if (!ok) break;  // warp-uniform: no tcgen05.ld of an accumulator that is not complete
-            tc_fence_after();
             int m, n;
             persist_tile(t, Mt, Nt, Bm, m, n);
             const int row = m * 128 + quarter * 32 + lane;
-            persist_epilogue<BN, EPI>(g, tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN), row, row < M, n);
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], u, err));
+            if (!ok) break;  // warp-uniform: no tcgen05.ld of an accumulator that is not complete
+            tc_fence_after();
+            const uint32_t tacc = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN);
+            if constexpr (EPI == EPI_RESID)
+                resid_add_tma(&tmC, boxes, tacc, BN, m * 128 + quarter * 32, n * BN, M, nbox);
+            else
+                persist_epilogue<BN, EPI>(g, tacc, row, row < M, n);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[b]);
         }
+        if (EPI == EPI_RESID && lane == 0) bulk_wait_all();  // reductions done before the CTA's memory goes
     }
     tc_fence_before();
     __syncthreads();
@@ -350,7 +418,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemmp_kernel(const __grid_constant_
 // waits.
 constexpr int kP2Stage = 2 * 128 * BK * 2;        // A 16 KB + B 16 KB per CTA
 constexpr int kP2Stages = 6;
-constexpr int kP2Smem = kP2Stages * kP2Stage + 1024;
+constexpr int kP2Smem = kP2Stages * kP2Stage + kResidStage + 1024;  // ring, residual staging, alignment slack
 constexpr uint32_t kP2TmemCols = 512;             // two 256-column accumulators
 
 __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t bar_cluster, void* dst, int x, int y) {
@@ -380,10 +448,14 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
+// tmC: the fp32 residual stream (box 32 columns x 32 rows, 128-byte swizzle), tmBt: the weights in 32-row
+// boxes, for the column slabs of a last partial round (both EPI_RESID only).
 template <int EPI>
 __global__ void __launch_bounds__(192, 1) tc_gemmp2_kernel(const __grid_constant__ CUtensorMap tmA,
                                                            const __grid_constant__ CUtensorMap tmB,
-                                                           const __grid_constant__ CUtensorMap tmB2, GemmArgs g,
+                                                           const __grid_constant__ CUtensorMap tmB2,
+                                                           const __grid_constant__ CUtensorMap tmC,
+                                                           const __grid_constant__ CUtensorMap tmBt, GemmArgs g,
                                                            int* err) {
     pdl_trigger();
     extern __shared__ uint8_t smem_raw[];
@@ -427,13 +499,40 @@ __global__ void __launch_bounds__(192, 1) tc_gemmp2_kernel(const __grid_constant
     }
     pdl_wait();
 
-    const int M = min(g.M_dev ? *g.M_dev : g.M_bound, g.M_bound);
+    const int live = min(g.M_dev ? *g.M_dev : g.M_bound, g.M_bound);
+    const int M = g.live_gate == kGateManyRows && live <= 256 ? 0 : live;  // 0: the few-row kernel's launch
     const int Mt = (M + 255) / 256;
     const int Nt = EPI == EPI_SWIGLU ? g.N / 128 : (g.N + 255) / 256;
     const int T = Mt * Nt;
     const int nk = g.K / BK;
     const int Bm = max(1, min(Mt, (int)(kBandBytes / ((size_t)256 * g.K * 2))));
     const int pair = blockIdx.x >> 1, pairs = gridDim.x >> 1;
+    // Work items: the full rounds' tiles, then the tiles of a last, partial round (all tiles, when there are
+    // fewer than pairs) cut into S column slabs of 256 / S columns (S = 4 or 2, the most that keeps one
+    // round; residual GEMMs only), so that the last round keeps more pairs busy.  A slab is computed whole
+    // (full K) by one pair: no partial sums.  Item w >= T_full is slab (w - T_full) % S of tile
+    // T_full + (w - T_full) / S.
+    int T_full = T, S = 1;
+    if (EPI == EPI_RESID) {
+        const int rem = T % pairs;
+        if (rem > 0) {
+            S = rem * 4 <= pairs ? 4 : rem * 2 <= pairs ? 2 : 1;
+            if (S > 1) T_full = T - rem;
+        }
+    }
+    const int W = T_full + (T - T_full) * S;
+    // tile, first column of the item within the tile, columns of the item
+    auto item = [&](int w, int& tile, int& c0, int& cw) {
+        if (w < T_full) {
+            tile = w;
+            c0 = 0;
+            cw = 256;
+        } else {
+            tile = T_full + (w - T_full) / S;
+            cw = 256 / S;
+            c0 = ((w - T_full) % S) * cw;
+        }
+    };
     const uint32_t full0 = cluster_map(smem_u32(&full_bar[0]), 0);      // the leader's full barriers
     const uint32_t empty0 = cluster_map(smem_u32(&acc_empty[0]), 0);    // the leader's accumulator-empty
 
@@ -442,9 +541,12 @@ __global__ void __launch_bounds__(192, 1) tc_gemmp2_kernel(const __grid_constant
             // ---- TMA producer of this rank's halves
             uint32_t q = 0;
             bool ok = true;
-            for (int t = pair; ok && t < T; t += pairs) {
-                int m, n;
+            for (int w = pair; ok && w < W; w += pairs) {
+                int t, c0, cw, m, n;
+                item(w, t, c0, cw);
                 persist_tile(t, Mt, Nt, Bm, m, n);
+                // a slab: each rank brings cw / 2 weight rows, in 32-row boxes
+                const uint32_t pair_bytes = cw == 256 ? 2u * kP2Stage : 2u * (kP2Stage / 2 + (uint32_t)cw / 2 * 128u);
                 for (int kb = 0; kb < nk; ++kb) {
                     const int s = (int)(q % kP2Stages);
                     const uint32_t ph = (q / kP2Stages) & 1u;
@@ -454,12 +556,16 @@ __global__ void __launch_bounds__(192, 1) tc_gemmp2_kernel(const __grid_constant
                     }
                     uint8_t* st = smem + s * kP2Stage;
                     const uint32_t fb = full0 + (uint32_t)(s * sizeof(uint64_t));
-                    if (leader) mbar_expect_tx(&full_bar[s], 2u * kP2Stage);  // the pair's bytes
+                    if (leader) mbar_expect_tx(&full_bar[s], pair_bytes);  // the pair's bytes
                     tma_load_2d_pair(&tmA, fb, st, kb * BK, m * 256 + (int)rank * 128);
                     if (EPI == EPI_SWIGLU)
                         tma_load_2d_pair(rank == 0 ? &tmB : &tmB2, fb, st + kP2Stage / 2, kb * BK, n * 128);
-                    else
+                    else if (cw == 256)
                         tma_load_2d_pair(&tmB, fb, st + kP2Stage / 2, kb * BK, n * 256 + (int)rank * 128);
+                    else
+                        for (int j = 0; j < cw / 64; ++j)
+                            tma_load_2d_pair(&tmBt, fb, st + kP2Stage / 2 + j * 32 * 128, kb * BK,
+                                             n * 256 + c0 + (int)rank * (cw / 2) + j * 32);
                     ++q;
                 }
             }
@@ -472,11 +578,14 @@ __global__ void __launch_bounds__(192, 1) tc_gemmp2_kernel(const __grid_constant
         if (lane == 0) {
             if (leader) {
                 // ---- MMA issuer for the pair (one thread of the leader)
-                constexpr uint32_t idesc = idesc_bf16(256, 256);
                 uint32_t q = 0;
                 int it = 0;
                 bool ok = true;
-                for (int t = pair; ok && t < T; t += pairs, ++it) {
+                for (int w = pair; ok && w < W; w += pairs, ++it) {
+                    int t, c0, cw;
+                    item(w, t, c0, cw);
+                    const uint32_t idesc = cw == 256 ? idesc_bf16(256, 256) : cw == 128 ? idesc_bf16(256, 128)
+                                                                                        : idesc_bf16(256, 64);
                     const int b = it & 1;
                     const uint32_t u = (uint32_t)(it >> 1) & 1u;
                     if (!mbar_wait(&acc_empty[b], u ^ 1u, err)) {
@@ -513,21 +622,32 @@ __global__ void __launch_bounds__(192, 1) tc_gemmp2_kernel(const __grid_constant
     } else {
         // ---- epilogue: this rank's 128 rows of the pair tile, one row per thread
         const int quarter = warp & 3;
+        const int r128 = quarter * 32 + lane;  // row within this rank's half of the tile
+        uint8_t* boxes = smem + kP2Stages * kP2Stage + quarter * 2 * kResidBox;  // EPI_RESID staging
+        uint32_t nbox = 0;
         int it = 0;
-        for (int t = pair; t < T; t += pairs, ++it) {
+        if (EPI == EPI_RESID && lane == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmC) : "memory");
+        for (int w = pair; w < W; w += pairs, ++it) {
+            int t, c0, cw, m, n;
+            item(w, t, c0, cw);
             const int b = it & 1;
             const uint32_t u = (uint32_t)(it >> 1) & 1u;
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], u, err));
-            if (!ok) break;
-            tc_fence_after();
-            int m, n;
             persist_tile(t, Mt, Nt, Bm, m, n);
-            const int row = m * 256 + (int)rank * 128 + quarter * 32 + lane;
-            persist_epilogue<256, EPI>(g, tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * 256), row, row < M, n);
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], u, err));
+            if (!ok) break;  // warp-uniform: no tcgen05.ld of an accumulator that is not complete
+            tc_fence_after();
+            const uint32_t tacc = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * 256);
+            if constexpr (EPI == EPI_RESID)
+                resid_add_tma(&tmC, boxes, tacc, cw, m * 256 + (int)rank * 128 + quarter * 32, n * 256 + c0, M,
+                                    nbox);
+            else
+                persist_epilogue<256, EPI>(g, tacc, m * 256 + (int)rank * 128 + r128, m * 256 + (int)rank * 128 + r128 < M,
+                                           n);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(empty0 + (uint32_t)(b * sizeof(uint64_t)));
         }
+        if (EPI == EPI_RESID && lane == 0) bulk_wait_all();  // reductions done before the CTA's memory goes
     }
     tc_fence_before();
     __syncthreads();

@@ -19,12 +19,16 @@ def _case(name="sdar1.7b_n32_b32"):
 def test_step_work_has_every_launch_of_the_step():
     # embedding + norm; per full layer QKV, attention, O, norm, gate/up, down (+ one norm between the two
     # full layers); selection; the gathering norm; per kept layer QKV, attention, O, norm, gate/up, down,
-    # norm; LM head; combine + decode; selection and the row map are two launches: 7 L + 6 launches
-    for name in ("sdar1.7b_n32_b32", "sdar8b_n256_b64", "small_bf16"):
+    # norm; LM head; combine + decode; selection and the row map are two launches: 7 L + 6 launches.
+    # With more than 256 kept-row slots (N x k_max) each kept-row GEMM and the LM head are two launches
+    # (few-row and many-row kernel, one of which exits on the live row count): 4 (L - 2) + 1 more
+    for name, few in (("sdar1.7b_n32_b32", True), ("sdar8b_n256_b64", False), ("small_bf16", True),
+                      ("sdar1.7b_n128_b32", False)):
         case = _case(name)
-        N = case.work.n_requests
+        N, L = case.work.n_requests, case.shape.n_layers
+        assert (N * case.work.k_max <= 256) == few
         work = bench.step_work(case, R=N, kept_per_req=[1] * N, plen=[64] * N)
-        assert sum(n for _, n, _, _ in work) == 7 * case.shape.n_layers + 6
+        assert sum(n for _, n, _, _ in work) == 7 * L + 6 + (0 if few else 4 * (L - 2) + 1)
 
 
 def test_kept_row_gemm_bytes_are_the_weights_plus_rows():
