@@ -217,9 +217,10 @@ __global__ void __launch_bounds__(t5_threads<QT>(), T5<QT>::kMinBlocks) attentio
                     if (!mbar_wait(&kv_empty[st], ((uint32_t)(i / kStages) & 1u) ^ 1u, a.err)) break;
                     valid_s[st] = issue_chunk(a, u, &pool_map, &ibc_map, kv_s + st * kStageBytes, &kv_full[st], i,
                                               n_prefix_chunks, pt);
-                    // kept-row units: ask L2 for the next chunk while it waits for a stage (the full-block
-                    // units' query tiles walk the same pages side by side and gain nothing from it, measured)
-                    if (!FULL && i + 1 >= kStages) prefetch_chunk_l2(a, u, i + 1, n_prefix_chunks, pt);
+                    // kept-row units of the two-CTAs-per-SM shape: ask L2 for the next chunk while it waits for
+                    // a stage (measured: the full-block units' query tiles walk the same pages side by side,
+                    // and the four-stage shape has its chunks in flight already; both lost time to it)
+                    if (!FULL && QT == 64 && i + 1 >= kStages) prefetch_chunk_l2(a, u, i + 1, n_prefix_chunks, pt);
                     ++issued;
                 }
                 // never leave with copies in flight
