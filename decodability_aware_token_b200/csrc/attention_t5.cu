@@ -150,21 +150,13 @@ __global__ void __launch_bounds__(t5_threads<QT>(), T5<QT>::kMinBlocks) attentio
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.Hq / a.Hkv;
     Unit u{};
-    // grid (query tiles, requests, KV heads): the query tiles of one unit run side by side, so the walks
-    // after the first find the unit's pages in L2
+    // grid (query tiles, KV heads, request slots): the query tiles of one unit run side by side (the walks
+    // after the first find the unit's pages in L2), and the CTAs of one request are adjacent.  With a
+    // request order (kept-row launches: longest prefix first, written by the row-map kernel earlier in
+    // the step) slot z walks request order[z], so the longest walks start first and the launch's tail is
+    // made of the shortest ones; the order is read after the programmatic-launch wait.
     u.qt = blockIdx.x;
-    u.b = blockIdx.y;
-    u.g = blockIdx.z;
-    u.P = checked_prefix(a.prefix_len, u.b, a.max_pages * a.page_size, a.err);
-    u.q0 = u.qt * QT;
-    const int n_prefix_chunks = (u.P + kChunk - 1) / kChunk;
-    const int n_chunks = n_prefix_chunks + 1;
-    const int unit = (u.b * a.Hkv + u.g) * q_tiles + u.qt;
-
-    const bool pt_cached = a.max_pages <= kPtCache;
-    for (int i = threadIdx.x; pt_cached && i < a.max_pages; i += blockDim.x)
-        pt_s[i] = a.page_table[(size_t)u.b * a.max_pages + i];
-    const int32_t* pt = pt_cached ? pt_s : a.page_table + (size_t)u.b * a.max_pages;
+    u.g = blockIdx.y;
 
     if (threadIdx.x == 0) {
         mbar_init(&q_full, 1);
@@ -194,6 +186,18 @@ __global__ void __launch_bounds__(t5_threads<QT>(), T5<QT>::kMinBlocks) attentio
     const uint32_t tmem = tmem_slot;
     pdl_wait();
 
+    u.b = a.order ? a.order[blockIdx.z] : (int)blockIdx.z;
+    u.P = checked_prefix(a.prefix_len, u.b, a.max_pages * a.page_size, a.err);
+    u.q0 = u.qt * QT;
+    const int n_prefix_chunks = (u.P + kChunk - 1) / kChunk;
+    const int n_chunks = n_prefix_chunks + 1;
+    const int unit = (u.b * a.Hkv + u.g) * q_tiles + u.qt;
+    const bool pt_cached = a.max_pages <= kPtCache;
+    for (int i = threadIdx.x; pt_cached && i < a.max_pages; i += blockDim.x)
+        pt_s[i] = a.page_table[(size_t)u.b * a.max_pages + i];
+    const int32_t* pt = pt_cached ? pt_s : a.page_table + (size_t)u.b * a.max_pages;
+    __syncthreads();  // the cached page-table row
+
     if (FULL) {
         u.row_base = u.b * a.B;
         u.n_rows = a.B;
@@ -220,7 +224,7 @@ __global__ void __launch_bounds__(t5_threads<QT>(), T5<QT>::kMinBlocks) attentio
                     // kept-row units of the two-CTAs-per-SM shape: ask L2 for the next chunk while it waits for
                     // a stage (measured: the full-block units' query tiles walk the same pages side by side,
                     // and the four-stage shape has its chunks in flight already; both lost time to it)
-                    if (!FULL && QT == 64 && i + 1 >= kStages) prefetch_chunk_l2(a, u, i + 1, n_prefix_chunks, pt);
+                    if (!FULL && QT == 64) prefetch_chunk_l2(a, u, i + 2, n_prefix_chunks, pt);  // two ahead
                     ++issued;
                 }
                 // never leave with copies in flight
@@ -484,7 +488,7 @@ template <int QT>
 int launch_t5(const AttnArgs& a, int q_tiles, const CUtensorMap& pool_map, const CUtensorMap& ibc_map, cudaStream_t s) {
     CUtensorMap q_map;
     if (!make_q_map(&q_map, a.q, a.q_rows_cap, a.Hq, a.Hq / a.Hkv, QT)) return -1;
-    const dim3 grid(q_tiles, a.N, a.Hkv), block(t5_threads<QT>());
+    const dim3 grid(q_tiles, a.Hkv, a.N), block(t5_threads<QT>());
     if (a.row_offsets == nullptr)
         return launched(launch_pdl(attention_t5_kernel<true, QT>, grid, block, t5_smem<QT>(), s, 0, pool_map, ibc_map,
                                    q_map, a, q_tiles));

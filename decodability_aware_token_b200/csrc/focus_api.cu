@@ -40,6 +40,7 @@ struct focus_ctx {
     double* inv_freq;
     float2* rope_tab;     // bf16 path: [rope_positions][head_dim / 2] (cos, sin)
     int32_t* masked_count;  // block loop: masked positions left after a step
+    int32_t* req_order;     // [max_requests] requests by descending prefix length (kept-row attention order)
     int* err;
     float *att_part_o, *att_part_ml, *att_sb;
     int* att_counters;
@@ -138,10 +139,11 @@ Layout plan(const focus_model_cfg* c, const focus_limits* l) {
         rows_c * 4, rows_c * 4,                             // 21-22 per-row confidence / top id
         split * rope_positions(l) * (size_t)c->head_dim / 2 * 8,  // 23 RoPE (cos, sin) table
         64,                                                 // 24 block loop: masked-position count
+        (size_t)l->max_requests * 4,                        // 25 request order
     };
     Layout lay{};
     size_t at = 0;
-    for (int i = 0; i < 25; ++i) {
+    for (int i = 0; i < 26; ++i) {
         lay.off[i] = at;
         at = align_up(at + sizes[i], 1024);
     }
@@ -291,6 +293,7 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
     sa.keep_count = out->keep_count; sa.retained_idx = out->retained_idx; sa.row_offsets = out->row_offsets;
     sa.importance_out = out->importance; sa.row_req = c->row_req; sa.row_pos = c->row_pos; sa.row_src = c->row_src;
     sa.n_rows = c->n_rows; sa.err = c->err;
+    sa.prefix_len = in->prefix_len; sa.max_prefix = max_prefix; sa.order = bf ? c->req_order : nullptr;
     run(FOCUS_K_SELECT, [&] { return launch_select(sa, s); });
     // ---- gather the kept rows (folding in layer 1's MLP partial sums) and normalise for layer 2
     const void* g_next = dm.L > 2 ? c->attn_norm[2] : c->final_norm;
@@ -316,6 +319,7 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
         at.q_rows = k_cap;
         at.row_offsets = out->row_offsets;
         at.imp_part = nullptr;
+        at.order = bf ? c->req_order : nullptr;  // longest prefix first (written by the row-map kernel)
         at.pieces = pieces_kept;
         run(FOCUS_K_ATTN_RAGGED, [&] { return attention(at, qt_kept); });
         gemm(FOCUS_K_GEMM_O, tc ? EPI_RESID : EPI_PARTIAL, c->o, c->wo[l], nullptr, R_bound, c->n_rows, dm.D,
@@ -443,6 +447,7 @@ int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_l
     c->inv_freq = reinterpret_cast<double*>(base + lay.off[15]);
     c->rope_tab = reinterpret_cast<float2*>(base + lay.off[23]);
     c->masked_count = reinterpret_cast<int32_t*>(base + lay.off[24]);
+    c->req_order = reinterpret_cast<int32_t*>(base + lay.off[25]);
     c->err = reinterpret_cast<int*>(base + lay.off[16]);
     c->att_part_o = reinterpret_cast<float*>(base + lay.off[17]);
     c->att_part_ml = reinterpret_cast<float*>(base + lay.off[18]);

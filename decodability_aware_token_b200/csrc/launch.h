@@ -96,6 +96,7 @@ struct AttnArgs {
     int* counters;              // [unit] arrival counters, zero between launches
     int q_rows;                 // bound on query rows per request in this launch (B, or the kept-row cap)
     int q_rows_cap;             // rows the query buffer holds
+    const int32_t* order;       // tcgen05 kernel: [N] request of each grid slot (null: slot b is request b)
 };
 
 constexpr int kAttnSplitCap = 1280;  // unit-pieces the split-KV scratch holds
@@ -132,6 +133,9 @@ struct SelectArgs {
     int32_t* row_src;           // [R_max] = b * B + j
     int32_t* n_rows;            // [1] = R
     int* err;
+    const int32_t* prefix_len;  // [N] (clamped to [0, max_prefix] for the order)
+    int max_prefix;
+    int32_t* order;             // [N] requests by descending prefix length, ties by index (null: not wanted)
 };
 int launch_select(const SelectArgs& a, cudaStream_t s);
 

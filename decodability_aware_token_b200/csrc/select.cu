@@ -169,6 +169,19 @@ __global__ void __launch_bounds__(1024) rowmap_kernel(SelectArgs a) {
             a.row_src[off + t] = b * a.B + j;
         }
     }
+    if (a.order) {
+        // requests by descending prefix length (ties by index): request b goes to the slot of its rank
+        auto len = [&](int b) { return min(max(a.prefix_len[b], 0), a.max_prefix); };
+        for (int b = tid; b < a.N; b += 1024) {
+            const int pb = len(b);
+            int rank = 0;
+            for (int c = 0; c < a.N; ++c) {
+                const int pc = len(c);
+                rank += (pc > pb || (pc == pb && c < b)) ? 1 : 0;
+            }
+            a.order[rank] = b;
+        }
+    }
 }
 
 }  // namespace
