@@ -90,9 +90,14 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_const
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.Hq / a.Hkv;
     Unit u{};
-    u.b = blockIdx.x;
-    u.g = blockIdx.y % a.Hkv;
-    u.qt = blockIdx.z;
+    // grid (KV heads x pieces, query tiles, request slots): a request's CTAs are adjacent.  With a request
+    // order (kept-row launches with more units than resident CTAs: longest prefix first, written by the
+    // row-map kernel earlier in the step), slot z walks request order[z], read after the wait; the early
+    // chunk copies below then also come after it.
+    if (a.order) pdl_wait();
+    u.b = a.order ? a.order[blockIdx.z] : (int)blockIdx.z;
+    u.g = blockIdx.x % a.Hkv;
+    u.qt = blockIdx.y;
     // Before the programmatic-launch wait this kernel reads only what no kernel of the step writes: the
     // prefix lengths, the page table and the prefix pages of the KV pool (the step's first kernel lets
     // its successors start only after everything queued before the step has completed).  The block's
@@ -104,7 +109,7 @@ __global__ void __launch_bounds__(128, 2) attention_tc_kernel(const __grid_const
     // split-KV: this CTA walks chunks [c_begin, c_end) of the unit's n_chunks
     const int pieces = a.pieces;  // grid.y = Hkv * pieces
     const int cpp = (n_chunks + pieces - 1) / pieces;  // chunks per piece
-    const int piece = blockIdx.y / a.Hkv;
+    const int piece = blockIdx.x / a.Hkv;
     const int c_begin = piece * cpp, c_end = min(n_chunks, c_begin + cpp);
     if (c_begin >= c_end) return;
     const int n_active = (n_chunks + cpp - 1) / cpp;
@@ -538,7 +543,7 @@ int launch_attention_tc(const AttnArgs& a, int q_tiles, cudaStream_t s) {
         pool_map = ibc_map;  // never used: with no pages every prefix key is invalid
     }
     const int smem = kAttnSmem;  // opted in by configure_attention_tc_kernels (at focus_init, per device)
-    dim3 grid(a.N, a.Hkv * a.pieces, q_tiles);
+    dim3 grid(a.Hkv * a.pieces, q_tiles, a.N);
     if (a.row_offsets == nullptr)
         return launched(launch_pdl(attention_tc_kernel<true>, grid, dim3(128), smem, s, 0, pool_map, ibc_map, a, q_tiles));
     return launched(launch_pdl(attention_tc_kernel<false>, grid, dim3(128), smem, s, 0, pool_map, ibc_map, a, q_tiles));

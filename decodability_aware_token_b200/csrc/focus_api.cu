@@ -26,6 +26,7 @@ struct focus_ctx {
     focus_model_cfg cfg;
     focus_limits lim;
     int device;
+    int sms;                // streaming multiprocessors of the device
     Dims dm;
     size_t elt;  // bytes per T
     // borrowed weights
@@ -319,7 +320,11 @@ int run_step(focus_ctx* c, const focus_batch* in, const focus_params* p, focus_s
         at.q_rows = k_cap;
         at.row_offsets = out->row_offsets;
         at.imp_part = nullptr;
-        at.order = bf ? c->req_order : nullptr;  // longest prefix first (written by the row-map kernel)
+        // longest prefix first (written by the row-map kernel) when the units outnumber the CTAs resident at
+        // once (two per SM); a single wave gains nothing and keeps the mma.sync kernel's early chunk copies
+        at.order = bf && (attention_t5_used(k_cap, dm.Hq / dm.Hkv) || N * dm.Hkv * qt_kept > 2 * c->sms)
+                       ? c->req_order
+                       : nullptr;
         at.pieces = pieces_kept;
         run(FOCUS_K_ATTN_RAGGED, [&] { return attention(at, qt_kept); });
         gemm(FOCUS_K_GEMM_O, tc ? EPI_RESID : EPI_PARTIAL, c->o, c->wo[l], nullptr, R_bound, c->n_rows, dm.D,
@@ -404,6 +409,10 @@ int focus_init(const focus_model_cfg* cfg, const focus_weights* w, const focus_l
     c->cfg = *cfg;
     c->lim = *lim;
     if (cudaGetDevice(&c->device) != cudaSuccess) {
+        delete c;
+        return FOCUS_ERR_CUDA;
+    }
+    if (cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
         delete c;
         return FOCUS_ERR_CUDA;
     }
