@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(t5_threads<QT>(), T5<QT>::kMinBlocks) attentio
                     // kept-row units of the two-CTAs-per-SM shape: ask L2 for the next chunk while it waits for
                     // a stage (measured: the full-block units' query tiles walk the same pages side by side,
                     // and the four-stage shape has its chunks in flight already; both lost time to it)
-                    if (!FULL && QT == 64) prefetch_chunk_l2(a, u, i + 2, n_prefix_chunks, pt);  // two ahead
+                    if (!FULL && QT == 64) prefetch_chunk_l2(a, u, i + 3, n_prefix_chunks, pt);  // three ahead
                     ++issued;
                 }
                 // never leave with copies in flight
